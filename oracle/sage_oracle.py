@@ -1,0 +1,387 @@
+"""CPU oracle for SageAttention2-style quantized attention (K/V smoothing, INT8 QK,
+FP8 PV, FP32 online softmax) on BF16 [B, N, H, D] ("NHD") tensors.
+
+TEST INFRASTRUCTURE ONLY.  Plain, slow and meant to be read against the method
+step by step.  Only the tests, the package smoke check and the benchmark's
+CPU-baseline leg may import it.  It shares no code with the CUDA library and
+imports nothing from it.
+
+Sources (page, section):
+* "FLUX.3 Action RTX 5090 report", 02 ENGINEERING, card 03 (SageAttention2):
+  INT8 QK, FP8 PV, FP32 accumulation, K smooth and V smooth kept, NHD layout.
+* same page, last-round card A: K centring (token mean subtracted) fused with
+  the INT8 quantization, keeping the original BF16 rounding of the centred K;
+  Q uses the same scale and INT8 rule.
+* same page, card C: V mean / scale / quant with V smoothing, V written in a
+  transposed, padded layout.
+* "MiniMax H3 on DGX Spark", 01 Precision map: Sage2++ = QK INT8 / PV FP8.
+* "为什么A10也能跑得动FLUX.1", 1.1: E4M3 = 4 exponent + 3 mantissa bits.
+
+The pages print no formula, block size or rounding rule.  The contract below
+(block of 64 tokens for Q/K scales, per-channel V scales, 128-key tiles, the
+rounding steps) is the plain reading stated with each function.  Every
+floating-point step that the GPU does in FP32 is rounded to FP32 here
+(``rn32``); exact integer dot products are formed in float64, which is exact
+for |sum| < 2**53.
+
+Parity status: pinned by tests/test_oracle_sage.py (quantizers by brute force
+and invariants; the attention tile loop by running it with quantization off
+against brute-force FP64 softmax attention; smoothing by the softmax shift
+invariance; closed forms for degenerate inputs).  The exp2 of the FP32 softmax
+is evaluated in FP64 and rounded once; the GPU's hardware exp2 is not
+bit-matched by design, which is why attention parity has a tolerance.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .numerics import (bf16_bits_to_f32, e4m3_decode, e4m3_encode,
+                       f32_to_bf16_bits, f64_to_bf16_bits, rn32,
+                       round_f32_to_bf16)
+
+QK_BLOCK = 64        # tokens per INT8 scale block of Q and K
+TILE = 128           # query rows per tile and keys per KV tile
+SUM_BLOCK = 64       # tokens per first-level FP64 partial sum
+SUM_LANES = 8        # interleaved second-level partial sums
+INT8_MAX = 127.0
+E4M3_MAX = 448.0
+LOG2E = 1.4426950408889634
+
+
+def npad(n: int) -> int:
+    """Padded token count: N rounded up to a whole 128-row tile."""
+    return ((n + TILE - 1) // TILE) * TILE
+
+
+# ----------------------------------------------------------------------------
+# A1 / A4: column sums over tokens in a fixed FP64 order
+# ----------------------------------------------------------------------------
+def column_sum_f64(x: np.ndarray) -> np.ndarray:
+    """Sum x[b, n, c] over n in FP64, in the contract's fixed order.
+
+    The pages only say "subtract the mean"; to make the means (and so every
+    code) reproducible the order of the FP64 additions is fixed:
+      1. 64-token blocks: s_c = ((0 + x_{64c}) + x_{64c+1}) + ... in token
+         order, over the block's tokens that exist (the last may be short);
+      2. 8 interleaved lanes: u_g = ((0 + s_g) + s_{g+8}) + s_{g+16} + ...;
+      3. butterfly over the lanes: for o in 4, 2, 1: u_g <- u_g + u_{g xor o};
+         the column sum is u_0.
+    Input x: float32 or float64 [B, N, C]; returns float64 [B, C].
+    """
+    x = np.asarray(x)
+    B, N, C = x.shape
+    nb = (N + SUM_BLOCK - 1) // SUM_BLOCK
+    partial = np.zeros((B, nb, C), dtype=np.float64)
+    for c in range(nb):
+        s = np.zeros((B, C), dtype=np.float64)
+        for n in range(c * SUM_BLOCK, min(N, (c + 1) * SUM_BLOCK)):
+            s = s + x[:, n, :].astype(np.float64)
+        partial[:, c] = s
+    lanes = np.zeros((B, SUM_LANES, C), dtype=np.float64)
+    for g in range(SUM_LANES):
+        u = np.zeros((B, C), dtype=np.float64)
+        for c in range(g, nb, SUM_LANES):
+            u = u + partial[:, c]
+        lanes[:, g] = u
+    idx = np.arange(SUM_LANES)
+    for o in (4, 2, 1):
+        lanes = lanes + lanes[:, idx ^ o]
+    return lanes[:, 0]
+
+
+# ----------------------------------------------------------------------------
+# A2: INT8 block quantization (Q as is, K after centring)
+# ----------------------------------------------------------------------------
+def int8_block_quant(x: np.ndarray):
+    """Quantize x[B, H, Npad, D] (float32, zero in padded rows) per 64-token block.
+
+    For each (b, h, block of 64 consecutive tokens, all D channels):
+      amax  = max |x| over the block,
+      scale = RN32(amax / 127),  inv = RN32(127 / amax),
+      code  = clamp(RNE(RN32(x * inv)), -127, 127);
+    amax == 0 gives scale = inv = 0 and all codes 0.
+    Returns (codes int8 [B, H, Npad, D], scale float32 [B, H, Npad/64]).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    B, H, Np, D = x.shape
+    xb = x.reshape(B, H, Np // QK_BLOCK, QK_BLOCK, D)
+    amax = np.max(np.abs(xb), axis=(3, 4))
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1))
+    scale = np.where(nz, safe / np.float32(INT8_MAX), np.float32(0)).astype(np.float32)
+    inv = np.where(nz, np.float32(INT8_MAX) / safe, np.float32(0)).astype(np.float32)
+    prod = (xb * inv[..., None, None]).astype(np.float32)
+    codes = np.clip(np.rint(prod), -INT8_MAX, INT8_MAX).astype(np.int8)
+    return codes.reshape(B, H, Np, D), scale
+
+
+def _nhd_to_bhnd_padded(x32: np.ndarray) -> np.ndarray:
+    B, N, H, D = x32.shape
+    out = np.zeros((B, H, npad(N), D), dtype=np.float32)
+    out[:, :, :N, :] = np.transpose(x32, (0, 2, 1, 3))
+    return out
+
+
+def k_mean_bf16(k_bits: np.ndarray) -> np.ndarray:
+    """A1: per-(b, h, d) token mean of K, FP64 sum, ONE rounding to BF16.
+
+    mean = RN_bf16(sum / N) with the sum in the fixed order of column_sum_f64
+    and the FP64 quotient rounded straight to BF16.  Returns uint16 [B, H, D].
+    """
+    B, N, H, D = k_bits.shape
+    k32 = bf16_bits_to_f32(k_bits).reshape(B, N, H * D)
+    s = column_sum_f64(k32)
+    return f64_to_bf16_bits(s / np.float64(N)).reshape(B, H, D)
+
+
+def quant_qk(q_bits: np.ndarray, k_bits: np.ndarray):
+    """A1-A3: K smoothing and INT8 block quantization of Q and K.
+
+    q_bits, k_bits: BF16 bit patterns uint16 [B, N, H, D].
+    K is centred by its BF16 token mean and rounded back to BF16 before
+    quantization:  kc = RN_bf16(RN32(k - mean_k)).  Q is quantized raw (the
+    pages keep only K and V smoothing).
+    Returns dict with q_codes, q_scale, k_codes, k_scale (layouts as
+    int8_block_quant) and k_mean (uint16 [B, H, D]).
+    """
+    q32 = bf16_bits_to_f32(q_bits)
+    k32 = bf16_bits_to_f32(k_bits)
+    mean_bits = k_mean_bf16(k_bits)
+    mean32 = bf16_bits_to_f32(mean_bits)                       # [B, H, D]
+    kc = round_f32_to_bf16((k32 - mean32[:, None, :, :]).astype(np.float32))
+    q_codes, q_scale = int8_block_quant(_nhd_to_bhnd_padded(q32))
+    k_codes, k_scale = int8_block_quant(_nhd_to_bhnd_padded(kc))
+    return dict(q_codes=q_codes, q_scale=q_scale, k_codes=k_codes,
+                k_scale=k_scale, k_mean=mean_bits)
+
+
+# ----------------------------------------------------------------------------
+# A4 / A5: V smoothing and per-channel FP8 quantization, transposed layout
+# ----------------------------------------------------------------------------
+def v_stats(v_bits: np.ndarray):
+    """A4: per-(b, h, d) mean, absmax of the centred V, and the FP8 scales.
+
+    mean  = RN32(sum / N)      (sum in the order of column_sum_f64)
+    amax  = max(RN32(vmax - mean), RN32(mean - vmin))  (= max |RN32(v - mean)|,
+            because rounding is monotone)
+    scale = RN32(amax / 448),  inv = RN32(448 / amax);  amax == 0 -> 0, 0.
+    Returns float32 arrays [B, H, D]: mean, amax, scale, inv.
+    """
+    B, N, H, D = v_bits.shape
+    v32 = bf16_bits_to_f32(v_bits).reshape(B, N, H * D)
+    mean = rn32(column_sum_f64(v32) / np.float64(N))
+    vmax = v32.max(axis=1)
+    vmin = v32.min(axis=1)
+    amax = np.maximum((vmax - mean).astype(np.float32), (mean - vmin).astype(np.float32))
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1))
+    scale = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(0)).astype(np.float32)
+    inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(0)).astype(np.float32)
+    shp = (B, H, D)
+    return (mean.reshape(shp), amax.reshape(shp), scale.reshape(shp), inv.reshape(shp))
+
+
+def quant_v(v_bits: np.ndarray):
+    """A4-A5: centre V per channel and quantize to E4M3 with per-channel scales.
+
+    vc = RN32(v - mean);  code = E4M3_RNE_satfinite(RN32(vc * inv)).
+    Codes are written transposed, [B, H, D, Npad], with zero codes for the
+    padded tokens N..Npad-1.
+    Returns dict with v_codes_t (uint8), v_scale, v_mean (float32 [B, H, D]).
+    """
+    B, N, H, D = v_bits.shape
+    mean, _, scale, inv = v_stats(v_bits)
+    v32 = bf16_bits_to_f32(v_bits)                               # [B, N, H, D]
+    vc = (v32 - mean[:, None, :, :]).astype(np.float32)
+    codes = e4m3_encode((vc * inv[:, None, :, :]).astype(np.float32))
+    out = np.zeros((B, H, D, npad(N)), dtype=np.uint8)
+    out[:, :, :, :N] = np.transpose(codes, (0, 2, 3, 1))
+    return dict(v_codes_t=out, v_scale=scale, v_mean=mean)
+
+
+# ----------------------------------------------------------------------------
+# A6-A10: tiled attention with FP32 online softmax
+# ----------------------------------------------------------------------------
+def _identity(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, quant_p,
+                 p_unit, two_pass=False):
+    """Online-softmax attention over 128-key tiles for one (b, h).
+
+    S         [R, >= n_keys] float64: exact score numerators (INT32 dot
+              products, or FP64 dot products with quantization off).
+    col_mult  f(j0, j1) -> [R, j1 - j0] multipliers taking S into the exp2
+              domain (dequant scales x sm_scale x log2 e).
+    Vt        [D, >= n_keys] float64: the (centred, dequantized-code) values.
+    out_mult  [D] per-channel output factor (V scale / p_unit); out_add [D]
+              the V mean added back.
+    rn        rounding applied after every step (rn32, or identity in FP64).
+    quant_p   P quantizer applied to p * p_unit (E4M3 round trip, or identity).
+
+    Per tile j (keys j0..j1-1, those >= n_keys excluded):
+      t     = rn(S * c)                          A7 dequant
+      m_new = max(m, max_k t)
+      alpha = rn(exp2(rn(m - m_new)))            (0 on the first tile)
+      p     = rn(exp2(rn(t - m_new)))            P~ in [0, 1]
+      l     = rn(rn(l * alpha) + rn(sum_k p))    row sum of UNquantized P~
+      P8    = quant_p(rn(p * p_unit))            A8
+      acc   = rn(rn(acc * alpha) + rn(P8 @ V))   A9, product sum exact then rounded
+    Epilogue (A10): o = rn(rn(rn(acc * out_mult) * rn(1 / l)) + out_add).
+    two_pass: m is the final row max from the start (alpha = 1 throughout).
+    Returns (o [R, D], m [R], l [R]).
+    """
+    R = S.shape[0]
+    D = Vt.shape[0]
+    nkv = (n_keys + TILE - 1) // TILE
+    m = np.full(R, -np.inf)
+    if two_pass:
+        for j in range(nkv):
+            j0, j1 = j * TILE, min(n_keys, (j + 1) * TILE)
+            t = rn(S[:, j0:j1] * col_mult(j0, j1))
+            m = np.maximum(m, t.max(axis=1))
+    l = np.zeros(R)
+    acc = np.zeros((R, D))
+    for j in range(nkv):
+        j0, j1 = j * TILE, min(n_keys, (j + 1) * TILE)
+        t = rn(S[:, j0:j1] * col_mult(j0, j1))
+        m_new = m if two_pass else np.maximum(m, t.max(axis=1))
+        with np.errstate(invalid="ignore"):
+            alpha = np.where(np.isneginf(m), 0.0, rn(np.exp2(rn(m - m_new))))
+        if two_pass:
+            alpha = np.ones(R)
+        p = rn(np.exp2(rn(t - m_new[:, None])))
+        l = rn(rn(l * alpha) + rn(p.sum(axis=1)))
+        p8 = quant_p(rn(p * p_unit))
+        acc = rn(rn(acc * alpha[:, None]) + rn(p8 @ Vt[:, j0:j1].T))
+        m = m_new
+    o = rn(rn(rn(acc * out_mult[None, :]) * rn(1.0 / l)[:, None]) + out_add[None, :])
+    return o, m, l
+
+
+def _e4m3_round_trip(x):
+    return e4m3_decode(e4m3_encode(np.asarray(x, dtype=np.float32)))
+
+
+def default_sm_scale(D: int) -> np.float32:
+    return np.float32(1.0 / math.sqrt(D))
+
+
+def exp2_scale(sm_scale) -> np.float32:
+    """sm_scale * log2(e), formed in FP64 from the FP32 sm_scale, rounded once."""
+    return np.float32(np.float64(np.float32(sm_scale)) * LOG2E)
+
+
+def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
+             sm_scale=None, rows=None, heads=None, two_pass=False, want_lse=False):
+    """A6-A10 on quantized operands; the output is the FP32 attention output.
+
+    q_codes, k_codes int8 [B, H, Npad, D]; q_scale, k_scale f32 [B, H, Npad/64];
+    v_codes_t uint8 E4M3 [B, H, D, Npad]; v_scale, v_mean f32 [B, H, D].
+    Score dequant multiplier for query row i and key j:
+        c = RN32(RN32(qs[i // 64] * ks[j // 64]) * RN32(sm_scale * log2 e)),
+    the P scale is 448 (P8 = E4M3(P~ * 448)) and the output factor is
+    RN32(v_scale / 448).  sm_scale None or <= 0 means 1/sqrt(D).
+    rows: optional query-row indices (< N) to evaluate; heads: optional list of
+    (b, h) pairs.  Returns float32 [B, R, H, D] (unevaluated heads stay 0),
+    plus lse [B, H, R] (natural log of the softmax denominator) if asked.
+    """
+    B, H, Np, D = q_codes.shape
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = default_sm_scale(D)
+    sl2e = exp2_scale(sm_scale)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    R = rows.shape[0]
+    out = np.zeros((B, R, H, D), dtype=np.float32)
+    lse = np.zeros((B, H, R), dtype=np.float32)
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    out_mult = None
+    for b, h in heads:
+        Qf = q_codes[b, h, rows].astype(np.float64)
+        Kf = k_codes[b, h, :N].astype(np.float64)
+        S = Qf @ Kf.T                                        # exact INT32 dots
+        qs = q_scale[b, h, rows // QK_BLOCK]
+        ks = k_scale[b, h]
+
+        def col_mult(j0, j1, qs=qs, ks=ks):
+            kk = ks[np.arange(j0, j1) // QK_BLOCK]
+            return rn32(rn32(qs[:, None].astype(np.float64) * kk[None, :]) * np.float64(sl2e))
+
+        Vt = e4m3_decode(v_codes_t[b, h, :, :N])
+        out_mult = rn32(np.float64(v_scale[b, h]) / E4M3_MAX)
+        o, m, l = _attend_rows(S, col_mult, Vt, out_mult.astype(np.float64),
+                               v_mean[b, h].astype(np.float64), N, rn32,
+                               _e4m3_round_trip, E4M3_MAX, two_pass=two_pass)
+        out[b, :, h, :] = o
+        lse[b, h] = rn32((m + np.log2(l)) * math.log(2.0))
+    return (out, lse) if want_lse else out
+
+
+def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
+                     smooth_v=True, heads=None):
+    """The same tile loop with quantization OFF, all in FP64.
+
+    q, k, v: float64 [B, N, H, D].  Scores are exact FP64 dot products, the
+    multiplier is sm_scale * log2 e, P is not quantized (p_unit 1), V is
+    centred by its FP64 mean (smooth_v) and K by its FP64 mean (smooth_k).
+    Used to pin the tile loop, the rescaling and the smoothing algebra against
+    brute-force softmax attention.  Returns float64 [B, R, H, D].
+    """
+    B, _, H, D = q.shape
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / math.sqrt(D)
+    c = sm_scale * LOG2E
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, rows.shape[0], H, D))
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in heads:
+        Q = q[b, rows, h, :]
+        K = k[b, :N, h, :]
+        if smooth_k:
+            K = K - K.mean(axis=0)
+        V = v[b, :N, h, :]
+        mean = V.mean(axis=0) if smooth_v else np.zeros(D)
+        S = Q @ K.T
+        o, _, _ = _attend_rows(S, lambda j0, j1: c, (V - mean).T, np.ones(D), mean,
+                               N, _identity, _identity, 1.0)
+        out[b, :, h, :] = o
+    return out
+
+
+def attn_exact_fp64(q, k, v, N, sm_scale=None, rows=None, heads=None):
+    """Plain softmax(Q K^T * sm_scale) V in FP64 on the given values, no tiling.
+
+    q, k, v: float64 [B, N, H, D].  Returns float64 [B, R, H, D].
+    """
+    B, _, H, D = q.shape
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / math.sqrt(D)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, rows.shape[0], H, D))
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in heads:
+        s = (q[b, rows, h, :] @ k[b, :N, h, :].T) * sm_scale
+        s = s - s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        out[b, :, h, :] = (e / e.sum(axis=1, keepdims=True)) @ v[b, :N, h, :]
+    return out
+
+
+def sage_pipeline(q_bits, k_bits, v_bits, sm_scale=None, rows=None, heads=None,
+                  two_pass=False):
+    """Whole path A1-A10 from BF16 inputs: returns (fp32 output, intermediates)."""
+    N = q_bits.shape[1]
+    qk = quant_qk(q_bits, k_bits)
+    vv = quant_v(v_bits)
+    o = attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"],
+                 vv["v_codes_t"], vv["v_scale"], vv["v_mean"], N, sm_scale=sm_scale,
+                 rows=rows, heads=heads, two_pass=two_pass)
+    return o, dict(qk, **vv)
+
+
+def bf16_output(o32: np.ndarray) -> np.ndarray:
+    """The BF16 output is the RNE rounding of the FP32 output (bit patterns)."""
+    return f32_to_bf16_bits(o32)
