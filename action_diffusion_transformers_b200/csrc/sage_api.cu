@@ -1,0 +1,392 @@
+// sage_api.cu - host side of the C ABI declared in include/sage.h.
+//
+// Validates every argument before launching, lays out the caller's workspace,
+// encodes the TMA tensor maps of the attention operands, launches the kernels
+// of sage_quant.cuh / sage_attn.cuh on the caller's stream and reports errors
+// as status codes with a thread-local message.  Nothing here allocates device
+// memory or synchronises, except sage_check().
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "sage.h"
+#include "sage_attn.cuh"
+#include "sage_quant.cuh"
+
+namespace {
+
+__device__ int g_sage_err;  // set to 1 by a kernel that gave up a bounded wait
+
+thread_local std::string g_last_error;
+std::atomic<int64_t> g_timeout_ns{2000000000LL};
+
+sage_status fail(sage_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+sage_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SAGE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  sage_status status = SAGE_OK;
+  std::string message;
+  int* err_ptr = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Once per device: check for sm_100, look up the error word, raise the shared
+// memory limit of the attention kernels, and find cuTensorMapEncodeTiled.
+sage_status device_setup(int* dev_out, int** err_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SAGE_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceState& ds = g_dev[dev];
+  if (!ds.ready) {
+    ds.ready = true;
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) {
+      ds.status = SAGE_ERR_CUDA;
+      ds.message = std::string("cudaGetDeviceProperties: ") + cudaGetErrorString(e);
+    } else if (prop.major != 10 || prop.minor != 0) {
+      ds.status = SAGE_ERR_UNSUPPORTED;
+      ds.message = "this library is built for sm_100a (B200); device is sm_" + std::to_string(prop.major) +
+                   std::to_string(prop.minor);
+    } else {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_sage_err);
+      if (e == cudaSuccess) {
+        ds.err_ptr = static_cast<int*>(p);
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::AttnSmem<128>::kAlloc);
+      }
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::AttnSmem<64>::kAlloc);
+      if (e == cudaSuccess && !g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e == cudaSuccess && (q != cudaDriverEntryPointSuccess || !fn)) e = cudaErrorSymbolNotFound;
+        if (e == cudaSuccess) g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+      if (e != cudaSuccess) {
+        ds.status = SAGE_ERR_CUDA;
+        ds.message = std::string("device setup: ") + cudaGetErrorString(e);
+      }
+    }
+  }
+  if (ds.status != SAGE_OK) return fail(ds.status, "%s", ds.message.c_str());
+  *dev_out = dev;
+  *err_out = ds.err_ptr;
+  return SAGE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t npad_of(int N) { return (static_cast<int64_t>(N) + 127) / 128 * 128; }
+
+// Shape checks shared by every call.  Host-only: runs without a GPU.
+sage_status check_shape(const sage_shape& s, int64_t* tok_stride) {
+  if (s.B < 1 || s.N < 1 || s.H < 1) return fail(SAGE_ERR_INVALID_ARG, "B, N, H must be >= 1 (got %d, %d, %d)", s.B, s.N, s.H);
+  if (s.D != 64 && s.D != 128) return fail(SAGE_ERR_UNSUPPORTED, "D must be 64 or 128 (got %d)", s.D);
+  const int64_t hd = static_cast<int64_t>(s.H) * s.D;
+  const int64_t ts = s.tok_stride == 0 ? hd : s.tok_stride;
+  if (ts < hd) return fail(SAGE_ERR_INVALID_ARG, "tok_stride %lld < H*D %lld", (long long)ts, (long long)hd);
+  if (ts % 8 != 0) return fail(SAGE_ERR_ALIGNMENT, "tok_stride %lld is not a multiple of 8", (long long)ts);
+  const int64_t np = npad_of(s.N);
+  if (static_cast<int64_t>(s.B) * s.H * np >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(s.B) * s.H * s.D >= (int64_t(1) << 31) || s.H > 65535 || 2LL * s.B > 65535)
+    return fail(SAGE_ERR_INVALID_ARG, "shape too large (B*H*Npad must stay below 2^31)");
+  if (s.cu_seqlens) {
+    if (s.n_seg < 1) return fail(SAGE_ERR_INVALID_ARG, "n_seg must be >= 1 with cu_seqlens");
+    if (s.cu_seqlens[0] != 0) return fail(SAGE_ERR_INVALID_ARG, "cu_seqlens[0] must be 0");
+    for (int i = 0; i < s.n_seg; ++i)
+      if (s.cu_seqlens[i + 1] < s.cu_seqlens[i])
+        return fail(SAGE_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing (index %d)", i + 1);
+    if (s.cu_seqlens[s.n_seg] != s.N)
+      return fail(SAGE_ERR_INVALID_ARG, "cu_seqlens[n_seg] = %d != N = %d", s.cu_seqlens[s.n_seg], s.N);
+  } else if (s.n_seg != 0) {
+    return fail(SAGE_ERR_INVALID_ARG, "n_seg = %d without cu_seqlens", s.n_seg);
+  }
+  *tok_stride = ts;
+  return SAGE_OK;
+}
+
+struct WsLayout {
+  size_t psum, pmin, pmax, kmean, vinv, total;
+};
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+WsLayout ws_layout(const sage_shape& s) {
+  const size_t nsb = (static_cast<size_t>(s.N) + sage::kSumBlock - 1) / sage::kSumBlock;
+  const size_t part = static_cast<size_t>(s.B) * nsb * s.H * s.D;
+  const size_t chans = static_cast<size_t>(s.B) * s.H * s.D;
+  WsLayout w;
+  w.psum = 0;
+  w.pmin = align256(w.psum + part * 8);
+  w.pmax = align256(w.pmin + part * 4);
+  w.kmean = align256(w.pmax + part * 4);
+  w.vinv = align256(w.kmean + chans * 2);
+  w.total = align256(w.vinv + chans * 4);
+  return w;
+}
+
+sage_status check_ws(const sage_shape& s, const void* ws, size_t ws_bytes, WsLayout* lay) {
+  *lay = ws_layout(s);
+  if (!ws) return fail(SAGE_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SAGE_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (ws_bytes < lay->total)
+    return fail(SAGE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, lay->total);
+  return SAGE_OK;
+}
+
+#define SAGE_NEED(p, name) \
+  do { if (!(p)) return fail(SAGE_ERR_INVALID_ARG, "%s is NULL", name); \
+       if (!aligned16(p)) return fail(SAGE_ERR_ALIGNMENT, "%s is not 16-byte aligned", name); } while (0)
+
+sage_status launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return SAGE_OK;
+}
+
+sage_status encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer, CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SAGE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return SAGE_OK;
+}
+
+template <int D>
+__global__ void selftest_wait_kernel(int64_t timeout_ns, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sage::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sage::fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the bounded wait must give up.
+  const bool ok = sage::mbar_wait_bounded(&bar, 0, reinterpret_cast<volatile int*>(&abort_flag), timeout_ns);
+  __syncthreads();
+  if (threadIdx.x == 0 && (!ok || abort_flag)) atomicExch(err, 1);
+  // Complete the barrier's phase so that no wait on it stays pending.
+  if (threadIdx.x == 0) sage::mbar_arrive(&bar);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sage_npad(int N) { return N < 1 ? 0 : static_cast<size_t>(npad_of(N)); }
+
+size_t sage_workspace_bytes(sage_shape s) {
+  int64_t ts;
+  if (check_shape(s, &ts) != SAGE_OK) return 0;
+  return ws_layout(s).total;
+}
+
+const char* sage_last_error(void) { return g_last_error.c_str(); }
+
+void sage_set_wait_timeout_ns(int64_t ns) { g_timeout_ns.store(ns > 0 ? ns : 2000000000LL); }
+
+sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_codes, float* q_scale,
+                          int8_t* k_codes, float* k_scale, void* k_mean, void* workspace, size_t ws_bytes,
+                          sage_stream_t stream) {
+  int64_t ts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  SAGE_NEED(q, "q");
+  SAGE_NEED(k, "k");
+  SAGE_NEED(q_codes, "q_codes");
+  SAGE_NEED(q_scale, "q_scale");
+  SAGE_NEED(k_codes, "k_codes");
+  SAGE_NEED(k_scale, "k_scale");
+  if (k_mean && !aligned16(k_mean)) return fail(SAGE_ERR_ALIGNMENT, "k_mean is not 16-byte aligned");
+  WsLayout lay;
+  if ((st = check_ws(s, workspace, ws_bytes, &lay)) != SAGE_OK) return st;
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* psum = reinterpret_cast<double*>(ws + lay.psum);
+  uint16_t* kmean = reinterpret_cast<uint16_t*>(ws + lay.kmean);
+  const int HD = s.H * s.D;
+  const int nsb = (s.N + sage::kSumBlock - 1) / sage::kSumBlock;
+  const int Npad = static_cast<int>(npad_of(s.N));
+  const uint16_t* qb = static_cast<const uint16_t*>(q);
+  const uint16_t* kb = static_cast<const uint16_t*>(k);
+
+  sage::colstats_partial<false><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum,
+                                                                                    nullptr, nullptr);
+  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
+                                                                static_cast<uint16_t*>(k_mean));
+  const dim3 g(Npad / sage::kQKBlock, s.H, 2 * s.B);
+  if (s.D == 128)
+    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  else
+    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  return launch_check("sage_quant_qk launch");
+}
+
+sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t, float* v_scale, float* v_mean,
+                         void* workspace, size_t ws_bytes, sage_stream_t stream) {
+  int64_t ts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  SAGE_NEED(v, "v");
+  SAGE_NEED(v_codes_t, "v_codes_t");
+  SAGE_NEED(v_scale, "v_scale");
+  SAGE_NEED(v_mean, "v_mean");
+  WsLayout lay;
+  if ((st = check_ws(s, workspace, ws_bytes, &lay)) != SAGE_OK) return st;
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* psum = reinterpret_cast<double*>(ws + lay.psum);
+  float* pmin = reinterpret_cast<float*>(ws + lay.pmin);
+  float* pmax = reinterpret_cast<float*>(ws + lay.pmax);
+  float* vinv = reinterpret_cast<float*>(ws + lay.vinv);
+  const int HD = s.H * s.D;
+  const int nsb = (s.N + sage::kSumBlock - 1) / sage::kSumBlock;
+  const int Npad = static_cast<int>(npad_of(s.N));
+  const uint16_t* vb = static_cast<const uint16_t*>(v);
+
+  sage::colstats_partial<true><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(vb, s.N, HD, ts, nsb, psum,
+                                                                                   pmin, pmax);
+  sage::v_stats_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, pmin, pmax, s.B, s.N, HD, nsb, v_mean,
+                                                                 v_scale, vinv);
+  const dim3 g(Npad / sage::kTile, s.H, s.B);
+  if (s.D == 128)
+    sage::v_quant_t<128><<<g, 256, 0, cs>>>(vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
+  else
+    sage::v_quant_t<64><<<g, 256, 0, cs>>>(vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
+  return launch_check("sage_quant_v launch");
+}
+
+sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
+                          const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
+                          const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32, float* lse,
+                          sage_stream_t stream) {
+  int64_t ts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  SAGE_NEED(q_codes, "q_codes");
+  SAGE_NEED(q_scale, "q_scale");
+  SAGE_NEED(k_codes, "k_codes");
+  SAGE_NEED(k_scale, "k_scale");
+  SAGE_NEED(v_codes_t, "v_codes_t");
+  SAGE_NEED(v_scale, "v_scale");
+  SAGE_NEED(v_mean, "v_mean");
+  SAGE_NEED(out, "out");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(SAGE_ERR_ALIGNMENT, "lse is not 4-byte aligned");
+  if (!(sm_scale == sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale is NaN");
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+
+  const int64_t Npad = npad_of(s.N);
+  const uint64_t rows = static_cast<uint64_t>(s.B) * s.H * Npad;
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle qk_swz = s.D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if ((st = encode_2d(&tq, q_codes, s.D, rows, s.D, sage::kBM, qk_swz)) != SAGE_OK) return st;
+  if ((st = encode_2d(&tk, k_codes, s.D, rows, s.D, sage::kBN, qk_swz)) != SAGE_OK) return st;
+  if ((st = encode_2d(&tv, v_codes_t, Npad, static_cast<uint64_t>(s.B) * s.H * s.D, sage::kBN, s.D,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK)
+    return st;
+
+    // sm_scale <= 0: 1/sqrt(D) formed in double and rounded once to float.
+  const float scale_f = sm_scale > 0.f ? sm_scale : static_cast<float>(1.0 / sqrt(static_cast<double>(s.D)));
+  const double scale = static_cast<double>(scale_f);
+  sage::AttnParams prm;
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
+  prm.v_scale = v_scale;
+  prm.v_mean = v_mean;
+  prm.out = out;
+  prm.lse = lse;
+  prm.err = err;
+  prm.N = s.N;
+  prm.H = s.H;
+  prm.Npad = static_cast<int>(Npad);
+  prm.nkv = static_cast<int>(Npad / sage::kBN);
+  prm.sl2e = static_cast<float>(scale * 1.4426950408889634);
+  prm.out_fp32 = out_fp32 ? 1 : 0;
+  prm.timeout_ns = g_timeout_ns.load();
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(Npad / sage::kBM), s.H, s.B);
+  if (s.D == 128)
+    sage::sage_attn_kernel<128><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+  else
+    sage::sage_attn_kernel<64><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+  return launch_check("sage_attn_fwd launch");
+}
+
+sage_status sage_check(sage_stream_t stream) {
+  int dev;
+  int* err;
+  sage_status st = device_setup(&dev, &err);
+  if (st != SAGE_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int flag = 0;
+  e = cudaMemcpy(&flag, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (flag) {
+    const int zero = 0;
+    e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    return fail(SAGE_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (timeout %lld ns)",
+                (long long)g_timeout_ns.load());
+  }
+  return SAGE_OK;
+}
+
+sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream) {
+  if (timeout_ns <= 0 || timeout_ns > 10000000000LL)
+    return fail(SAGE_ERR_INVALID_ARG, "timeout_ns must be in (0, 1e10]");
+  int dev;
+  int* err;
+  sage_status st = device_setup(&dev, &err);
+  if (st != SAGE_OK) return st;
+  selftest_wait_kernel<0><<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns, err);
+  return launch_check("selftest launch");
+}
+
+}  // extern "C"

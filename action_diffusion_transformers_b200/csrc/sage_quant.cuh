@@ -1,0 +1,359 @@
+// sage_quant.cuh - bandwidth-bound kernels of sage_quant_qk / sage_quant_v.
+//
+//  colstats_partial  per 64-token block, per channel: FP64 sum in token order
+//                    (and, for V, min / max) -> workspace partials.
+//  k_mean_finalize   FP64 block partials -> K mean, BF16 (one rounding).
+//  v_stats_finalize  FP64 block partials -> V mean, per-channel FP8 scales.
+//  qk_block_quant    Q and K (centred, BF16-rounded) -> INT8 codes with one
+//                    FP32 scale per 64-token block of one head.
+//  v_quant_t         centred V -> E4M3 codes, transposed through shared memory
+//                    to [B, H, D, Npad].
+//
+// All inputs are BF16 [B, N, H, D] with a token stride; every global access is
+// a 16-byte vector for the inputs.  Reductions use a fixed order, so repeated
+// calls give identical bytes.
+#pragma once
+#include "sage_ptx.cuh"
+
+namespace sage {
+
+constexpr int kQKBlock = 64;     // tokens per INT8 scale block
+constexpr int kSumBlock = 64;    // tokens per first-level FP64 partial
+constexpr int kSumLanes = 32;    // interleaved second-level partials
+constexpr int kTile = 128;       // padding granularity of the token axis
+
+__device__ __forceinline__ uint4 ld_nc_16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& raw, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+    f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Per (b, 64-token block c, channel): s = ((0 + x_{64c}) + x_{64c+1}) + ... in
+// token order, in FP64.  Grid (nsb, B, ceil(HD / (8*blockDim))).
+// ----------------------------------------------------------------------------
+template <bool kMinMax>
+__global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restrict__ x, int N, int HD,
+                                                        int64_t tok_stride, int nsb,
+                                                        double* __restrict__ psum,
+                                                        float* __restrict__ pmin, float* __restrict__ pmax) {
+  const int c = blockIdx.x;
+  const int b = blockIdx.y;
+  const int ch0 = (blockIdx.z * blockDim.x + threadIdx.x) * 8;
+  if (ch0 >= HD) return;
+  const int n0 = c * kSumBlock;
+  const int n1 = min(N, n0 + kSumBlock);
+  const uint16_t* p = x + (static_cast<int64_t>(b) * N + n0) * tok_stride + ch0;
+  double s[8];
+  float mn[8], mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s[i] = 0.0;
+    mn[i] = __int_as_float(0x7F800000);
+    mx[i] = -__int_as_float(0x7F800000);
+  }
+  int n = n0;
+  for (; n + 8 <= n1; n += 8) {
+    uint4 raw[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) raw[t] = ld_nc_16(p + static_cast<int64_t>(n - n0 + t) * tok_stride);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      float f[8];
+      unpack8(raw[t], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        s[i] = __dadd_rn(s[i], static_cast<double>(f[i]));
+        if (kMinMax) {
+          mn[i] = fminf(mn[i], f[i]);
+          mx[i] = fmaxf(mx[i], f[i]);
+        }
+      }
+    }
+  }
+  for (; n < n1; ++n) {
+    float f[8];
+    unpack8(ld_nc_16(p + static_cast<int64_t>(n - n0) * tok_stride), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      s[i] = __dadd_rn(s[i], static_cast<double>(f[i]));
+      if (kMinMax) {
+        mn[i] = fminf(mn[i], f[i]);
+        mx[i] = fmaxf(mx[i], f[i]);
+      }
+    }
+  }
+  const int64_t o = (static_cast<int64_t>(b) * nsb + c) * HD + ch0;
+  double2* ps = reinterpret_cast<double2*>(psum + o);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ps[i] = make_double2(s[2 * i], s[2 * i + 1]);
+  if (kMinMax) {
+    float4* pn = reinterpret_cast<float4*>(pmin + o);
+    float4* px = reinterpret_cast<float4*>(pmax + o);
+    pn[0] = make_float4(mn[0], mn[1], mn[2], mn[3]);
+    pn[1] = make_float4(mn[4], mn[5], mn[6], mn[7]);
+    px[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+    px[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
+  }
+}
+
+// Second level of the fixed summation order for one channel: lane g sums
+// blocks g, g+32, g+64, ... in increasing order from +0; then the butterfly
+// u_g <- u_g + u_{g^o} for o = 16, 8, 4, 2, 1; the result is lane 0's value.
+// Block of 1024 threads = 32 lanes (warps) x 32 channels (lanes of a warp, so
+// every load is one coalesced 256-byte row of partials); the channel index
+// runs over B*HD.  For V the same pass also reduces min / max (order-free).
+template <bool kMinMax>
+__device__ __forceinline__ void finalize_channel(const double* __restrict__ psum,
+                                                 const float* __restrict__ pmin,
+                                                 const float* __restrict__ pmax, int nsb, int HD, int b,
+                                                 int ch, bool valid, double (*sh)[33], float (*shn)[33],
+                                                 float (*shx)[33], double& sum, float& vmin, float& vmax) {
+  const int g = threadIdx.x >> 5;
+  const int cl = threadIdx.x & 31;
+  double u = 0.0;
+  float mn = __int_as_float(0x7F800000), mx = -__int_as_float(0x7F800000);
+  if (valid) {
+    const int64_t base = static_cast<int64_t>(b) * nsb * HD + ch;
+#pragma unroll 4
+    for (int c = g; c < nsb; c += kSumLanes) {
+      u = __dadd_rn(u, psum[base + static_cast<int64_t>(c) * HD]);
+      if (kMinMax) {
+        mn = fminf(mn, pmin[base + static_cast<int64_t>(c) * HD]);
+        mx = fmaxf(mx, pmax[base + static_cast<int64_t>(c) * HD]);
+      }
+    }
+  }
+  sh[g][cl] = u;
+  if (kMinMax) {
+    shn[g][cl] = mn;
+    shx[g][cl] = mx;
+  }
+  __syncthreads();
+  // Butterfly across the 32 lanes, every thread computing its own lane g.
+#pragma unroll
+  for (int o = kSumLanes / 2; o >= 1; o >>= 1) {
+    const double w = __dadd_rn(sh[g][cl], sh[g ^ o][cl]);
+    float wn = 0.f, wx = 0.f;
+    if (kMinMax) {
+      wn = fminf(shn[g][cl], shn[g ^ o][cl]);
+      wx = fmaxf(shx[g][cl], shx[g ^ o][cl]);
+    }
+    __syncthreads();
+    sh[g][cl] = w;
+    if (kMinMax) {
+      shn[g][cl] = wn;
+      shx[g][cl] = wx;
+    }
+    __syncthreads();
+  }
+  sum = sh[0][cl];
+  if (kMinMax) {
+    vmin = shn[0][cl];
+    vmax = shx[0][cl];
+  }
+}
+
+__global__ void __launch_bounds__(1024) k_mean_finalize(const double* __restrict__ psum, int B, int N, int HD,
+                                                        int nsb, uint16_t* __restrict__ mean_ws,
+                                                        uint16_t* __restrict__ mean_out) {
+  __shared__ double sh[kSumLanes][33];
+  const int gch = blockIdx.x * 32 + (threadIdx.x & 31);
+  const bool valid = gch < B * HD;
+  const int b = valid ? gch / HD : 0;
+  const int ch = valid ? gch % HD : 0;
+  double s = 0.0;
+  float dummy0, dummy1;
+  finalize_channel<false>(psum, nullptr, nullptr, nsb, HD, b, ch, valid, sh, nullptr, nullptr, s, dummy0,
+                          dummy1);
+  if (valid && threadIdx.x < 32) {
+    const uint16_t m = static_cast<uint16_t>(double_to_bf16_bits(__ddiv_rn(s, static_cast<double>(N))));
+    mean_ws[gch] = m;
+    if (mean_out) mean_out[gch] = m;
+  }
+}
+
+// V: mean = RN_f32(sum / N); amax = max(RN(vmax - mean), RN(mean - vmin));
+// scale = RN(amax / 448), inv = RN(448 / amax) (0, 0 for amax == 0).
+__global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restrict__ psum,
+                                                         const float* __restrict__ pmin,
+                                                         const float* __restrict__ pmax, int B, int N, int HD,
+                                                         int nsb, float* __restrict__ v_mean,
+                                                         float* __restrict__ v_scale, float* __restrict__ v_inv) {
+  __shared__ double sh[kSumLanes][33];
+  __shared__ float shn[kSumLanes][33];
+  __shared__ float shx[kSumLanes][33];
+  const int gch = blockIdx.x * 32 + (threadIdx.x & 31);
+  const bool valid = gch < B * HD;
+  const int b = valid ? gch / HD : 0;
+  const int ch = valid ? gch % HD : 0;
+  double s = 0.0;
+  float vmin = 0.f, vmax = 0.f;
+  finalize_channel<true>(psum, pmin, pmax, nsb, HD, b, ch, valid, sh, shn, shx, s, vmin, vmax);
+  if (valid && threadIdx.x < 32) {
+    const float mean = __double2float_rn(__ddiv_rn(s, static_cast<double>(N)));
+    const float amax = fmaxf(__fsub_rn(vmax, mean), __fsub_rn(mean, vmin));
+    float scale = 0.f, inv = 0.f;
+    if (amax > 0.f) {
+      scale = __fdiv_rn(amax, 448.f);
+      inv = __fdiv_rn(448.f, amax);
+    }
+    v_mean[gch] = mean;
+    v_scale[gch] = scale;
+    v_inv[gch] = inv;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// INT8 block quantization.  CTA = one (b, h, 64-token block) of Q (z even) or
+// K (z odd, centred by mean_k and rounded to BF16 first).  256 threads: D/8
+// threads cover one token row (8 channels each), 256/(D/8) rows per pass.
+// Grid (Npad/64, H, 2*B).
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict__ q,
+                                                      const uint16_t* __restrict__ k, int N, int H, int Npad,
+                                                      int64_t tok_stride, const uint16_t* __restrict__ k_mean,
+                                                      int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+                                                      int8_t* __restrict__ k_codes,
+                                                      float* __restrict__ k_scale) {
+  constexpr int kLPR = D / 8;             // threads per token row
+  constexpr int kRPP = 256 / kLPR;        // token rows per pass
+  constexpr int kTPT = kQKBlock / kRPP;   // tokens per thread
+  __shared__ float red[8];
+  const int blk = blockIdx.x;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z >> 1;
+  const bool is_k = blockIdx.z & 1;
+  const uint16_t* src = is_k ? k : q;
+  const int cg = threadIdx.x % kLPR;
+  const int r0 = threadIdx.x / kLPR;
+  const int d0 = cg * 8;
+
+  float mean[8];
+  if (is_k) {
+    const uint4 mraw = *reinterpret_cast<const uint4*>(k_mean + (static_cast<int64_t>(b) * H + h) * D + d0);
+    unpack8(mraw, mean);
+  }
+  float x[kTPT][8];
+  float amax = 0.f;
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int n = blk * kQKBlock + r0 + t * kRPP;
+    if (n < N) {
+      const uint4 raw = ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0);
+      unpack8(raw, x[t]);
+      if (is_k) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[t][i] = bf16_bits_to_float(float_to_bf16_bits(__fsub_rn(x[t][i], mean[i])));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[t][i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[t][i]));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  float scale = 0.f, inv = 0.f;
+  if (amax > 0.f) {
+    scale = __fdiv_rn(amax, 127.f);
+    inv = __fdiv_rn(127.f, amax);
+  }
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  int8_t* dst = is_k ? k_codes : q_codes;
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int n = blk * kQKBlock + r0 + t * kRPP;
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int c = __float2int_rn(__fmul_rn(x[t][i], inv));
+      c = max(-127, min(127, c));
+      w[i >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w[0], w[1]);
+  }
+  if (threadIdx.x == 0) (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + blk] = scale;
+}
+
+// ----------------------------------------------------------------------------
+// V centre + E4M3 quantization + transpose.  CTA = one (b, h, 128-token tile).
+// Phase 1: threads read 16-byte pieces of token rows, quantize 8 channels and
+// store the 8 code bytes into a [128][D] shared tile.  Phase 2: each thread
+// gathers 16 consecutive tokens of one channel and writes them as one 16-byte
+// piece of the transposed output row.  Grid (Npad/128, H, B).
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v, int N, int H, int Npad,
+                                                 int64_t tok_stride, const float* __restrict__ v_mean,
+                                                 const float* __restrict__ v_inv, uint8_t* __restrict__ out) {
+  constexpr int kLPR = D / 8;
+  constexpr int kRPP = 256 / kLPR;
+  constexpr int kTPT = kTile / kRPP;
+  constexpr int kPitch = D + 16;          // bytes per token row of the shared tile
+  __shared__ __align__(16) uint8_t tile[kTile * kPitch];
+  const int n0 = blockIdx.x * kTile;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int cg = threadIdx.x % kLPR;
+  const int r0 = threadIdx.x / kLPR;
+  const int d0 = cg * 8;
+  const int64_t bhd = (static_cast<int64_t>(b) * H + h) * D;
+  float mean[8], inv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    mean[i] = v_mean[bhd + d0 + i];
+    inv[i] = v_inv[bhd + d0 + i];
+  }
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int nl = r0 + t * kRPP;
+    const int n = n0 + nl;
+    uint32_t w0 = 0u, w1 = 0u;
+    if (n < N) {
+      float f[8];
+      unpack8(ld_nc_16(v + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0), f);
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fsub_rn(f[i], mean[i]), inv[i]);
+      w0 = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
+      w1 = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
+    }
+    *reinterpret_cast<uint2*>(tile + nl * kPitch + d0) = make_uint2(w0, w1);
+  }
+  __syncthreads();
+  constexpr int kChunks = D * (kTile / 16);  // 16-token pieces of all channel rows
+  for (int idx = threadIdx.x; idx < kChunks; idx += 256) {
+    const int d = idx % D;
+    const int qc = idx / D;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t acc = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc |= static_cast<uint32_t>(tile[(qc * 16 + j * 4 + i) * kPitch + d]) << (8 * i);
+      w[j] = acc;
+    }
+    *reinterpret_cast<uint4*>(out + (bhd + d) * Npad + n0 + qc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace sage

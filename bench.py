@@ -1,0 +1,335 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized-attention hot path on B200.
+
+One step = sage_quant_qk + sage_quant_v + sage_attn_fwd over one batch of the
+action-DiT joint-block workload (B=2 CFG cond/uncond, H=24, N=4096, D=128,
+BF16 NHD; synthetic, seeded).  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload action_dit|mid_video|long_video|ragged|tiny]
+
+value      = attention ops (4*B*H*N^2*D, INT8 QK^T + FP8 PV) per step, all ranks,
+             / device time of the whole step (quant + attention), in TOPS;
+             inputs resident in HBM, L2 flushed (256 MiB write) between steps,
+             per-step CUDA events on the launching stream, max over ranks.
+e2e        = the same metric through the Python API with pinned host inputs:
+             H2D of Q, K, V + the three calls + D2H of the BF16 output, per step.
+roofline   = the attention kernel alone: ops / its mean event-timed duration,
+             against the INT8/FP8 dense peak derived from the measured BF16 peak.
+cpu_baseline (N=1, rank 0) = the CPU oracle timed on a bounded sample.
+--impl reference runs the oracle (the reference arm of this build) instead.
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
+(replicas, weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 4.5 / 2.25  # nominal dense INT8/FP8 : BF16 tensor throughput ratio
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="action_dit", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def quant_bytes(w):
+    """Algorithmic bytes of the two quantization calls (per step)."""
+    elems = w.B * w.N * w.H * w.D
+    blocks = w.B * w.H * ((w.N + 127) // 128 * 2)
+    chans = w.B * w.H * w.D
+    qk = elems * (2 + 2 + 1 + 1) + blocks * 4 * 2 + chans * 2
+    v = elems * (2 + 1) + chans * 8
+    return qk, v
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.path = None
+        if gpu_id is None:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.count(",") >= 8]
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(dev_index: int):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev_index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[dev_index]
+        return str(dev_index)
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(w, qb, kb, vb, rows: int, heads: int):
+    """Time the CPU oracle on `heads` heads of batch 0 (full quantization of those
+    heads, attention for `rows` query rows).  Returns (ops, seconds)."""
+    from oracle import sage_oracle as so
+    t0 = time.perf_counter()
+    sl = (slice(0, 1), slice(None), slice(0, heads), slice(None))
+    qk = so.quant_qk(qb[sl], kb[sl])
+    vv = so.quant_v(vb[sl])
+    r = synth.sample_rows(w.N, rows, 0)[:rows] if rows < w.N else None
+    so.attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"], vv["v_codes_t"], vv["v_scale"],
+                vv["v_mean"], w.N, rows=r)
+    dt = time.perf_counter() - t0
+    nrows = w.N if r is None else len(r)
+    return 4.0 * heads * nrows * w.N * w.D, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    qb, kb, vb = synth.generate(w)
+    rows, heads = 256, 1
+    for _ in range(args.warmup):
+        oracle_sample(w, qb, kb, vb, rows, heads)
+    times = []
+    ops = 0.0
+    for _ in range(args.steps):
+        ops, dt = oracle_sample(w, qb, kb, vb, rows, heads)
+        times.append(dt)
+    tot = sum(times)
+    value = ops * len(times) / tot / 1e12
+    sample = f"1 head of batch 0: full K/V quantization of that head + attention for {rows} query rows"
+    line = {"impl": "reference", "metric": "quantized-attention TOPS", "value": value, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D},
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- ours
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import action_diffusion_transformers_b200 as adt
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = synth.WORKLOADS[args.workload]
+    qb, kb, vb = synth.generate(w)
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
+    q, k, v = as_dev(qb), as_dev(kb), as_dev(vb)
+    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def quant_qk():
+        adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                          buf.workspace, stream)
+
+    def quant_v():
+        adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
+
+    def attn():
+        adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
+                          buf.v_mean, buf.shape, 0.0, buf.out, False, None, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        quant_qk(); quant_v(); attn()
+    adt.sage_check()
+    torch.cuda.synchronize()
+    barrier()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(gpu_id_for(local))
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        e = ev[i]
+        e[0].record(stream)
+        quant_qk()
+        e[1].record(stream)
+        quant_v()
+        e[2].record(stream)
+        attn()
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    adt.sage_check()
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+    qk_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    v_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    at_ms = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ops = w.attn_ops
+    value = world * ops * K / (max_total_ms / 1e3) / 1e12
+
+    # --------------------------------------------------------------- e2e (host buffers)
+    pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
+    hq, hk, hv = pin(qb), pin(kb), pin(vb)
+    hout = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for _ in range(2):
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        quant_qk(); quant_v(); attn()
+        hout.copy_(buf.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        e2e_ev[i][0].record(stream)
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
+        quant_qk(); quant_v(); attn()
+        hout.copy_(buf.out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    adt.sage_check()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * ops * K / (float(t.item()) / 1e3) / 1e12
+    h2d = 3 * qb.nbytes
+    d2h = buf.out.numel() * buf.out.element_size()
+
+    # --------------------------------------------------------------- roofline, baseline
+    peaks, src = load_peaks()
+    peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    attn_mean_ms = statistics.mean(at_ms)
+    achieved = ops / (attn_mean_ms / 1e3) / 1e12
+    qk_bytes, v_bytes = quant_bytes(w)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows, heads = 512, 2
+        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads)
+        cpu = {"value": o_ops / o_dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{heads} heads of batch 0: full K/V quantization of those heads + attention for "
+                         f"{rows} query rows each ({o_dt:.1f} s)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "quantized-attention TOPS", "value": value, "unit": "TOPS", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_total_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "global_batch": w.B * world,
+                   "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "sage_attn_kernel<128>",
+                     "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"},
+        "kernels_us": {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
+                       "attn": 1e3 * attn_mean_ms},
+        "quant_gbs": {"quant_qk": qk_bytes / (statistics.mean(qk_ms) / 1e3) / 1e9,
+                      "quant_v": v_bytes / (statistics.mean(v_ms) / 1e3) / 1e9,
+                      "peak_hbm_gbs": peaks["hbm_gbs"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 7 * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * sage.h - C ABI of the B200 (sm_100a) quantized-attention library.
+ *
+ * The method (SageAttention2-style attention inside FLUX.3-Action and MiniMax-H3
+ * DiT blocks) is described on these pages:
+ *  - "FLUX.3 Action RTX 5090 report", 02 ENGINEERING, card 03 "SageAttention2":
+ *    INT8 QK, FP8 PV, FP32 accumulation, K smooth and V smooth kept, NHD layout;
+ *    and the last-round cards A (K centring fused into the INT8 quantization,
+ *    keeping the BF16 rounding of the centred K; Q quantized with the same
+ *    scale and INT8 rule) and C (V mean / scale / quant with V smoothing, V
+ *    read in place from a wider projection output and written transposed and
+ *    padded).
+ *  - "MiniMax H3 on DGX Spark", 01 Precision map: Sage2++ = QK INT8 / PV FP8.
+ *  - "为什么A10也能跑得动FLUX.1", 1.1: FP8 E4M3 = 4 exponent + 3 mantissa bits.
+ * The pages give no formulas; the contract fixed here (64-token Q/K scale
+ * blocks, per-channel V scales, 128-key tiles, rounding rules) is stated with
+ * each call.
+ *
+ * Conventions for every call:
+ *  - Tensors are device pointers owned by the caller.  The library never
+ *    allocates or frees memory; scratch space is the caller's workspace.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and never synchronise.  Device-side wait timeouts are
+ *    reported by sage_check().
+ *  - Arguments are validated on the host before any launch.  On an invalid
+ *    argument nothing is launched, the call returns a non-zero sage_status,
+ *    and sage_last_error() describes the problem (thread-local string).
+ *  - Device pointers must be 16-byte aligned; padded rows/columns of every
+ *    output are written (zero codes, zero scales) so outputs are fully defined.
+ *  - Results are deterministic: fixed launch configurations, fixed reduction
+ *    order, no atomics on values.
+ *
+ * Shapes: B batch, N tokens, H heads, D head dim (64 or 128).
+ * Npad = sage_npad(N) = N rounded up to a multiple of 128.
+ * BF16 inputs are [B, N, H, D] ("NHD"): element (b, n, h, d) sits at
+ * b*N*tok_stride + n*tok_stride + h*D + d, tok_stride >= H*D (0 means H*D),
+ * tok_stride a multiple of 8.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* sage_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, bad cu_seqlens   */
+  SAGE_ERR_UNSUPPORTED = 2,    /* D not 64/128, or no sm_100 device          */
+  SAGE_ERR_ALIGNMENT = 3,      /* pointer or stride alignment                */
+  SAGE_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed          */
+  SAGE_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up a bounded wait            */
+  SAGE_ERR_WORKSPACE = 6       /* workspace missing or smaller than needed   */
+} sage_status;
+
+typedef struct {
+  int B, N, H, D;
+  int64_t tok_stride;         /* elements between consecutive tokens of the
+                                 call's BF16 input(s); 0 means H*D           */
+  const int32_t* cu_seqlens;  /* HOST pointer to n_seg+1 segment offsets of a
+                                 packed joint sequence, or NULL.  Validated
+                                 (starts at 0, non-decreasing, ends at N) and
+                                 otherwise informational: attention is full
+                                 over the concatenation and the K/V means run
+                                 over all N tokens.                          */
+  int n_seg;
+} sage_shape;
+
+/* N rounded up to a whole 128-row tile. */
+SAGE_API size_t sage_npad(int N);
+
+/* Bytes of device workspace needed by sage_quant_qk and sage_quant_v for this
+ * shape (one buffer serves both; calls on one stream may share it). */
+SAGE_API size_t sage_workspace_bytes(sage_shape s);
+
+/*
+ * sage_quant_qk - K smoothing and INT8 block quantization of Q and K.
+ * ("FLUX.3 Action RTX 5090 report", last-round card A; card 03.)
+ *
+ * in : q, k        BF16 [B, N, H, D] with s.tok_stride (both tensors).
+ * out: q_codes     int8 [B, H, Npad, D]; rows >= N are 0.
+ *      q_scale     f32  [B, H, Npad/64]; blocks past N are 0.
+ *      k_codes     int8 [B, H, Npad, D]; k_scale f32 [B, H, Npad/64].
+ *      k_mean      BF16 [B, H, D] or NULL.
+ * Rule: mean_k[b,h,d] = RN_bf16(sum_n k / N), the FP64 sum taken in a fixed
+ * order (64-token blocks in token order; 32 interleaved lanes over blocks;
+ * butterfly 16,8,4,2,1 over lanes) and the quotient rounded once to BF16;
+ * kc = RN_bf16(RN_f32(k - mean_k)).  For each 64-token block of one (b,h)
+ * over all D: amax = max|x|, scale = RN(amax/127), inv = RN(127/amax),
+ * code = clamp(RNE(RN(x*inv)), -127, 127); amax == 0 gives 0 scale and codes.
+ * Q is quantized as is, K after centring.  Codes are bit-exact with that rule.
+ * workspace: >= sage_workspace_bytes(s) bytes of device memory, 256-B aligned.
+ */
+SAGE_API sage_status sage_quant_qk(const void* q, const void* k, sage_shape s,
+                          int8_t* q_codes, float* q_scale,
+                          int8_t* k_codes, float* k_scale, void* k_mean,
+                          void* workspace, size_t ws_bytes, sage_stream_t stream);
+
+/*
+ * sage_quant_v - V smoothing and per-channel FP8 E4M3 quantization, written
+ * transposed.  ("FLUX.3 Action RTX 5090 report", last-round card C; card 03.)
+ *
+ * in : v           BF16 [B, N, H, D] with s.tok_stride (may be a strided
+ *                  slice of a wider projection output).
+ * out: v_codes_t   E4M3 bytes [B, H, D, Npad]; tokens >= N are 0.
+ *      v_scale     f32 [B, H, D]; v_mean f32 [B, H, D].
+ * Rule: mean = RN_f32(sum/N) (FP64 sum, same order as sage_quant_qk);
+ * amax = max(RN(vmax - mean), RN(mean - vmin)); scale = RN(amax/448),
+ * inv = RN(448/amax) (0, 0 when amax == 0);
+ * code = E4M3_RNE_satfinite(RN(RN(v - mean) * inv)).  Bit-exact with that rule.
+ */
+SAGE_API sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t,
+                         float* v_scale, float* v_mean,
+                         void* workspace, size_t ws_bytes, sage_stream_t stream);
+
+/*
+ * sage_attn_fwd - O = softmax(Q K^T * sm_scale) V on the quantized operands.
+ * ("FLUX.3 Action RTX 5090 report", card 03: INT8 QK, FP8 PV, FP32
+ * accumulation, V mean added back; "MiniMax H3 on DGX Spark", 01.)
+ *
+ * in : the outputs of sage_quant_qk / sage_quant_v for the same shape
+ *      (s.tok_stride is ignored here).
+ *      sm_scale <= 0 selects 1/sqrt(D).
+ * out: out   [B, N, H, D], BF16 (out_fp32 == 0) or FP32 (out_fp32 != 0).
+ *      lse   f32 [B, H, N] natural-log softmax denominator, or NULL.
+ * Per 128-row query tile and 128-key tile: S = Qc Kc^T exactly in INT32 on the
+ * tensor cores; t = S * qs * ks * sm_scale * log2(e) in FP32; running row max m;
+ * P~ = exp2(t - m) in [0, 1]; l accumulates unquantized P~; P8 = E4M3(P~*448);
+ * O_acc = O_acc * exp2(m_old - m_new) + P8 V8 (FP8 MMA, FP32 accumulation);
+ * O = O_acc * (v_scale/448) / l + v_mean.  Keys >= N are masked.  Matches the
+ * contract within tolerance (hardware exp2 and MMA summation order).
+ */
+SAGE_API sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale,
+                          const int8_t* k_codes, const float* k_scale,
+                          const uint8_t* v_codes_t, const float* v_scale,
+                          const float* v_mean, sage_shape s, float sm_scale,
+                          void* out, int out_fp32, float* lse,
+                          sage_stream_t stream);
+
+/* Synchronises `stream`, then reports and clears a device-side wait timeout
+ * raised by any kernel of this library (SAGE_ERR_DEVICE_TIMEOUT), or a CUDA
+ * error (SAGE_ERR_CUDA); SAGE_OK otherwise. */
+SAGE_API sage_status sage_check(sage_stream_t stream);
+
+/* Bound, in nanoseconds, on every wait inside the library's kernels (default
+ * 2e9).  After it the kernel stops its work, drains its own copies and tensor
+ * operations, releases tensor memory, records a timeout for sage_check() and
+ * returns.  Values <= 0 restore the default. */
+SAGE_API void sage_set_wait_timeout_ns(int64_t ns);
+
+/* Failure-detection self-test: launches one CTA that waits on a barrier that
+ * nothing completes, bounded by timeout_ns; afterwards sage_check() returns
+ * SAGE_ERR_DEVICE_TIMEOUT and the context stays usable. */
+SAGE_API sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream);
+
+/* Message describing the last non-OK status of this thread. */
+SAGE_API const char* sage_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H_ */

@@ -44,7 +44,7 @@ from .numerics import (bf16_bits_to_f32, e4m3_decode, e4m3_encode,
 QK_BLOCK = 64        # tokens per INT8 scale block of Q and K
 TILE = 128           # query rows per tile and keys per KV tile
 SUM_BLOCK = 64       # tokens per first-level FP64 partial sum
-SUM_LANES = 8        # interleaved second-level partial sums
+SUM_LANES = 32       # interleaved second-level partial sums
 INT8_MAX = 127.0
 E4M3_MAX = 448.0
 LOG2E = 1.4426950408889634
@@ -65,9 +65,9 @@ def column_sum_f64(x: np.ndarray) -> np.ndarray:
     code) reproducible the order of the FP64 additions is fixed:
       1. 64-token blocks: s_c = ((0 + x_{64c}) + x_{64c+1}) + ... in token
          order, over the block's tokens that exist (the last may be short);
-      2. 8 interleaved lanes: u_g = ((0 + s_g) + s_{g+8}) + s_{g+16} + ...;
-      3. butterfly over the lanes: for o in 4, 2, 1: u_g <- u_g + u_{g xor o};
-         the column sum is u_0.
+      2. 32 interleaved lanes: u_g = ((0 + s_g) + s_{g+32}) + s_{g+64} + ...;
+      3. butterfly over the lanes: for o in 16, 8, 4, 2, 1:
+         u_g <- u_g + u_{g xor o}; the column sum is u_0.
     Input x: float32 or float64 [B, N, C]; returns float64 [B, C].
     """
     x = np.asarray(x)
@@ -86,8 +86,10 @@ def column_sum_f64(x: np.ndarray) -> np.ndarray:
             u = u + partial[:, c]
         lanes[:, g] = u
     idx = np.arange(SUM_LANES)
-    for o in (4, 2, 1):
+    o = SUM_LANES // 2
+    while o >= 1:
         lanes = lanes + lanes[:, idx ^ o]
+        o //= 2
     return lanes[:, 0]
 
 

@@ -13,8 +13,20 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: full-size workload parity (minutes)")
 
 
+def ensure_built():
+    """Build libsage.so if a source is newer (loads build.py by path, so the
+    package, which loads the library, is not imported first)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_sage_build", os.path.join(ROOT, "action_diffusion_transformers_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
 @pytest.fixture(scope="session")
-def lib():
-    """The CUDA library binding; GPU tests fail loudly when it is missing."""
-    import action_diffusion_transformers_b200 as adt
-    return adt
+def adt():
+    """The CUDA library binding; it raises ImportError when libsage.so is missing."""
+    ensure_built()
+    import action_diffusion_transformers_b200 as m
+    return m

@@ -1,0 +1,92 @@
+"""The C-ABI library on the host (no GPU needed): it loads, exports every call
+declared in include/sage.h, sizes its workspace, and rejects invalid
+arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "sage.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(adt):
+    names = _declared_functions()
+    assert {"sage_quant_qk", "sage_quant_v", "sage_attn_fwd"} <= set(names)
+    lib = ctypes.CDLL(adt.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(adt.EXPORTED)
+
+
+def test_npad_and_workspace(adt):
+    assert [adt.npad(n) for n in (1, 127, 128, 129, 4096, 55296)] == [128, 128, 128, 256, 4096, 55296]
+    assert adt.npad(0) == 0
+    s = adt.make_shape(2, 4096, 24, 128)
+    ws = adt.workspace_bytes(s)
+    nsb = 4096 // 64
+    assert ws >= 2 * nsb * 24 * 128 * 16 and ws % 256 == 0
+    assert adt.workspace_bytes(adt.make_shape(1, 100, 2, 96)) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first or no GPU is reached
+
+
+def _qk(adt, shape, **over):
+    a = dict(q=FAKE, k=FAKE, qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE, km=None, ws=0x100000, wsb=1 << 40)
+    a.update(over)
+    return adt._lib.sage_quant_qk(a["q"], a["k"], shape, a["qc"], a["qs"], a["kc"], a["ks"], a["km"], a["ws"],
+                                  a["wsb"], None)
+
+
+@pytest.mark.parametrize("B,N,H,D,ts,status", [
+    (1, 256, 2, 96, 0, 2),       # unsupported head dim
+    (1, 0, 2, 64, 0, 1),         # empty sequence
+    (0, 16, 2, 64, 0, 1),        # empty batch
+    (1, 16, 2, 64, 100, 1),      # token stride below H*D
+    (1, 16, 2, 64, 132, 3),      # token stride not a multiple of 8
+])
+def test_shape_validation(adt, B, N, H, D, ts, status):
+    assert _qk(adt, adt.make_shape(B, N, H, D, ts)) == status
+    assert adt._lib.sage_last_error()
+
+
+def test_pointer_validation(adt):
+    s = adt.make_shape(1, 256, 2, 64)
+    assert _qk(adt, s, q=None) == 1
+    assert _qk(adt, s, kc=FAKE + 8) == 3
+    assert _qk(adt, s, km=FAKE + 2) == 3
+    assert _qk(adt, s, ws=None) == 6
+    assert _qk(adt, s, ws=0x100010) == 3
+    assert _qk(adt, s, wsb=16) == 6
+    assert b"workspace" in adt._lib.sage_last_error()
+
+
+def test_cu_seqlens_validation(adt):
+    ok = adt.make_shape(1, 20480, 24, 128, cu_seqlens=[0, 512, 18944, 20448, 20480])
+    bad_end = adt.make_shape(1, 20480, 24, 128, cu_seqlens=[0, 512, 18944, 20448, 20479])
+    bad_order = adt.make_shape(1, 20480, 24, 128, cu_seqlens=[0, 512, 400, 20480])
+    bad_start = adt.make_shape(1, 20480, 24, 128, cu_seqlens=[3, 20480])
+    for s in (bad_end, bad_order, bad_start):
+        assert _qk(adt, s) == 1
+    # valid arguments get past validation; without a GPU the device lookup fails
+    st = _qk(adt, ok)
+    assert st in (0, 4)
+
+
+def test_attn_and_v_validation(adt):
+    s = adt.make_shape(1, 256, 2, 64)
+    L = adt._lib
+    assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, None, 0, None, None) == 1
+    assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, float("nan"), FAKE, 0, None, None) == 1
+    assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, FAKE, 0, FAKE + 2, None) == 3
+    assert L.sage_quant_v(FAKE, s, None, FAKE, FAKE, 0x100000, 1 << 40, None) == 1
+    assert L.sage_quant_v(FAKE, adt.make_shape(1, 256, 2, 128, 200), FAKE, FAKE, FAKE, 0x100000, 1 << 40,
+                          None) == 1
+    assert L.sage_selftest_wait_timeout(0, None) == 1
