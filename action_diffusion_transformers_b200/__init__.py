@@ -30,7 +30,9 @@ SAGE_OK = 0
 STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED", 3: "SAGE_ERR_ALIGNMENT",
                 4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_DEVICE_TIMEOUT", 6: "SAGE_ERR_WORKSPACE"}
 EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
-            "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error")
+            "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error",
+            "sage_quant_qk_static")
+QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class SageShape(ctypes.Structure):
@@ -46,6 +48,8 @@ _lib.sage_workspace_bytes.argtypes = [SageShape]
 _lib.sage_workspace_bytes.restype = ctypes.c_size_t
 _lib.sage_quant_qk.argtypes = [_vp, _vp, SageShape, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_qk.restype = ctypes.c_int
+_lib.sage_quant_qk_static.argtypes = [_vp, _vp, SageShape, _vp, _vp, _vp, _vp, _vp, _vp]
+_lib.sage_quant_qk_static.restype = ctypes.c_int
 _lib.sage_quant_v.argtypes = [_vp, SageShape, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_v.restype = ctypes.c_int
 _lib.sage_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, SageShape, ctypes.c_float, _vp, ctypes.c_int,
@@ -111,6 +115,15 @@ def sage_quant_qk(q, k, shape, q_codes, q_scale, k_codes, k_scale, k_mean, works
     ws_bytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
     _ok(_lib.sage_quant_qk(_ptr(q), _ptr(k), shape, _ptr(q_codes), _ptr(q_scale), _ptr(k_codes), _ptr(k_scale),
                            _ptr(k_mean), _ptr(workspace), ws_bytes, _stream(stream)), "sage_quant_qk")
+
+
+def sage_quant_qk_static(q, k, shape, q_codes, q_scale, k_codes, k_scale, k_mean, stream=None):
+    """sage_quant_qk without a workspace: for callers that cannot allocate
+    device memory.  Scratch lives in a fixed 8 MiB array inside the library;
+    larger shapes raise SageError (SAGE_ERR_WORKSPACE).  Calls that overlap on
+    the GPU share that array and race."""
+    _ok(_lib.sage_quant_qk_static(_ptr(q), _ptr(k), shape, _ptr(q_codes), _ptr(q_scale), _ptr(k_codes),
+                                  _ptr(k_scale), _ptr(k_mean), _stream(stream)), "sage_quant_qk_static")
 
 
 def sage_quant_v(v, shape, v_codes_t, v_scale, v_mean, workspace, stream=None):

@@ -207,6 +207,30 @@ __global__ void selftest_wait_kernel(int64_t timeout_ns, int* err) {
 
 }  // namespace
 
+// Scratch of sage_quant_qk_static: one array per GPU that loads the library.
+static __device__ __align__(256) unsigned char g_qk_static_scratch[SAGE_QK_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+unsigned char* g_qk_static_ptr[kMaxDevices];
+std::mutex g_qk_static_mu;
+
+// Device address of g_qk_static_scratch on the current device (looked up once
+// per device; host code only holds a stand-in for the array's name).
+sage_status qk_static_scratch(int dev, unsigned char** out) {
+  std::lock_guard<std::mutex> lock(g_qk_static_mu);
+  if (!g_qk_static_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_qk_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    g_qk_static_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_qk_static_ptr[dev];
+  return SAGE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t sage_npad(int N) { return N < 1 ? 0 : static_cast<size_t>(npad_of(N)); }
@@ -387,6 +411,55 @@ sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream)
   if (st != SAGE_OK) return st;
   selftest_wait_kernel<0><<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns, err);
   return launch_check("selftest launch");
+}
+
+
+sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int8_t* q_codes, float* q_scale,
+                                 int8_t* k_codes, float* k_scale, void* k_mean, sage_stream_t stream) {
+  int64_t ts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  SAGE_NEED(q, "q");
+  SAGE_NEED(k, "k");
+  SAGE_NEED(q_codes, "q_codes");
+  SAGE_NEED(q_scale, "q_scale");
+  SAGE_NEED(k_codes, "k_codes");
+  SAGE_NEED(k_scale, "k_scale");
+  if (k_mean && !aligned16(k_mean)) return fail(SAGE_ERR_ALIGNMENT, "k_mean is not 16-byte aligned");
+  const size_t nsb_sz = (static_cast<size_t>(s.N) + sage::kSumBlock - 1) / sage::kSumBlock;
+  const size_t chans = static_cast<size_t>(s.B) * s.H * s.D;
+  const size_t psum_bytes = align256(chans * nsb_sz * 8);
+  const size_t need = psum_bytes + align256(chans * 2);
+  if (need > SAGE_QK_STATIC_SCRATCH_BYTES)
+    return fail(SAGE_ERR_WORKSPACE,
+                "sage_quant_qk_static: shape needs %zu bytes of scratch, the built-in array holds %u; "
+                "use sage_quant_qk with a workspace",
+                need, SAGE_QK_STATIC_SCRATCH_BYTES);
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+  unsigned char* scratch = nullptr;
+  if ((st = qk_static_scratch(dev, &scratch)) != SAGE_OK) return st;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  double* psum = reinterpret_cast<double*>(scratch);
+  uint16_t* kmean = reinterpret_cast<uint16_t*>(scratch + psum_bytes);
+  const int HD = s.H * s.D;
+  const int nsb = static_cast<int>(nsb_sz);
+  const int Npad = static_cast<int>(npad_of(s.N));
+  const uint16_t* qb = static_cast<const uint16_t*>(q);
+  const uint16_t* kb = static_cast<const uint16_t*>(k);
+  // Every scratch byte read below is written earlier in the same call.
+  sage::colstats_partial<false><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum,
+                                                                                    nullptr, nullptr);
+  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
+                                                                static_cast<uint16_t*>(k_mean));
+  const dim3 g(Npad / sage::kQKBlock, s.H, 2 * s.B);
+  if (s.D == 128)
+    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  else
+    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  return launch_check("sage_quant_qk_static launch");
 }
 
 }  // extern "C"

@@ -165,6 +165,33 @@ SAGE_API void sage_set_wait_timeout_ns(int64_t ns);
  * SAGE_ERR_DEVICE_TIMEOUT and the context stays usable. */
 SAGE_API sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream);
 
+/*
+ * sage_quant_qk_static - sage_quant_qk without a workspace argument, for
+ * callers that cannot allocate device memory: a plugin whose host framework
+ * owns all device memory and offers no scratch hook, a runtime whose memory
+ * budget is fixed at start-up, or code that must not call cudaMalloc /
+ * cudaFree because those calls synchronise the device.  (The pages have no
+ * counterpart; this is an interface variant, not a step of the method.)
+ *
+ * Same inputs, outputs and rule as sage_quant_qk, bit-identical results.  The
+ * scratch (FP64 partial sums and the K mean) lives in one array inside the
+ * library, SAGE_QK_STATIC_SCRATCH_BYTES (8 MiB) per GPU that loads the
+ * library, held until the process exits.  Shapes whose scratch,
+ * B*ceil(N/64)*H*D*8 + B*H*D*2 bytes (each part rounded up to 256), exceeds
+ * it are rejected with SAGE_ERR_WORKSPACE before any launch.
+ * The call allocates nothing.  Its first call on a device looks up the
+ * array's device address (with that device current); make that first call
+ * before any stream capture.  Every call on a device shares the one array and
+ * it keeps the last call's contents (nothing in it needs to start at zero):
+ * calls that overlap on the GPU (concurrent streams) race on it, so order
+ * them on one stream or with events.
+ */
+#define SAGE_QK_STATIC_SCRATCH_BYTES (8u << 20)
+SAGE_API sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s,
+                                          int8_t* q_codes, float* q_scale,
+                                          int8_t* k_codes, float* k_scale, void* k_mean,
+                                          sage_stream_t stream);
+
 /* Message describing the last non-OK status of this thread. */
 SAGE_API const char* sage_last_error(void);
 
