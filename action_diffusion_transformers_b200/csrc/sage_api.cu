@@ -47,6 +47,7 @@ struct DeviceState {
   sage_status status = SAGE_OK;
   std::string message;
   int* err_ptr = nullptr;
+  int sm_count = 0;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -58,7 +59,7 @@ EncodeTiledFn g_encode = nullptr;
 
 // Once per device: check for sm_100, look up the error word, raise the shared
 // memory limit of the attention kernels, and find cuTensorMapEncodeTiled.
-sage_status device_setup(int* dev_out, int** err_out) {
+sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -77,6 +78,7 @@ sage_status device_setup(int* dev_out, int** err_out) {
       ds.message = "this library is built for sm_100a (B200); device is sm_" + std::to_string(prop.major) +
                    std::to_string(prop.minor);
     } else {
+      ds.sm_count = prop.multiProcessorCount;
       void* p = nullptr;
       e = cudaGetSymbolAddress(&p, g_sage_err);
       if (e == cudaSuccess) {
@@ -103,6 +105,7 @@ sage_status device_setup(int* dev_out, int** err_out) {
   if (ds.status != SAGE_OK) return fail(ds.status, "%s", ds.message.c_str());
   *dev_out = dev;
   *err_out = ds.err_ptr;
+  if (sm_count_out) *sm_count_out = ds.sm_count;
   return SAGE_OK;
 }
 
@@ -343,7 +346,8 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   if (!(sm_scale == sm_scale)) return fail(SAGE_ERR_INVALID_ARG, "sm_scale is NaN");
   int dev;
   int* err;
-  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+  int sm_count = 0;
+  if ((st = device_setup(&dev, &err, &sm_count)) != SAGE_OK) return st;
 
   const int64_t Npad = npad_of(s.N);
   const uint64_t rows = static_cast<uint64_t>(s.B) * s.H * Npad;
@@ -375,6 +379,7 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   prm.timeout_ns = g_timeout_ns.load();
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(static_cast<unsigned>(Npad / sage::kBM), s.H, s.B);
+  (void)sm_count;
   if (s.D == 128)
     sage::sage_attn_kernel<128><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
   else

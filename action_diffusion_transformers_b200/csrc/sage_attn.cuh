@@ -1,10 +1,17 @@
 // sage_attn.cuh - quantized attention forward on sm_100a tensor cores.
 //
 // One CTA computes one 128-row query tile of one (b, h).  Warp roles:
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
-//              TMEM, runs the FP32 online softmax, writes P as E4M3 into a
-//              128B-swizzled shared tile, rescales the O accumulator in TMEM
-//              when its row max moves, and runs the epilogue.
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Per tile it
+//              reads S from TMEM twice (row max, then exponentials 64 keys at a
+//              time, so only 64 scores are ever live in registers), writes P as
+//              E4M3 into a 128B-swizzled shared tile, rescales the O
+//              accumulator in TMEM when its row max moves, and runs the
+//              epilogue.  Two CTAs share an SM; their softmax warps are
+//              independent, so their MUFU-heavy and ALU-heavy phases interleave.
+// S is accumulated onto the integer 0x4B400000 (the bits of 1.5 * 2^23) that
+// the softmax warps write into the S columns before each QK^T MMA: read as a
+// float, a loaded S word is then exactly 1.5 * 2^23 + S (|S| <= 127^2 * D <
+// 2^22), so one exact subtraction converts it, two at a time with f32x2.
 //   warp 4     producer: one thread issues TMA tile loads (Q once; K and V
 //              tiles into 2-stage rings).
 //   warp 5     MMA: allocates TMEM; one thread issues
@@ -31,8 +38,18 @@ namespace sage {
 
 constexpr int kBM = 128;   // query rows per tile
 constexpr int kBN = 128;   // keys per tile
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 192;      // 4 softmax warps + producer + MMA
+constexpr int kSoftmaxThreads = 128;   // one thread per query row
+constexpr int kWarpProducer = 4;
+constexpr int kWarpMma = 5;
 constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSBiasBits = 0x4B400000u;   // S accumulates onto these bits
+constexpr float kSBias = 12582912.0f;          // their float value, 1.5 * 2^23
+constexpr float kLog2P8 = 8.8073549220576041f; // log2(448): the row sum holds 448 * P~
+#ifndef SAGE_POLY_PAIRS
+#define SAGE_POLY_PAIRS 0                      // of every 16 column pairs, exp2 on the FMA pipe
+#endif
+constexpr int kPolyPairs = SAGE_POLY_PAIRS;
 
 template <int D>
 struct AttnSmem {
@@ -46,7 +63,7 @@ struct AttnSmem {
   static constexpr int kV0 = kK1 + kKBytes;
   static constexpr int kV1 = kV0 + kVBytes;
   static constexpr int kP = kV1 + kVBytes;
-  static constexpr int kVf = kP + kPBytes;     // D floats: v_scale / 448
+  static constexpr int kVf = kP + kPBytes;     // D floats: v_scale
   static constexpr int kVm = kVf + 4 * D;      // D floats: v_mean
   static constexpr int kBar = kVm + 4 * D;     // 16 mbarriers
   static constexpr int kMisc = kBar + 16 * 8;  // tmem slot, abort flag
@@ -83,8 +100,105 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
   return __int2float_rn(static_cast<int>(s));
 }
 
+// One 32-column chunk of a score row, with the contract's rounding steps:
+// t = RN(S * c), u = RN(t - m_new), p = 2^u, y = RN(p * 448) -> E4M3 code;
+// the row sum accumulates y (= 448 * P~).  Only the exp2 itself differs from
+// the contract (hardware ex2.approx, or the FMA-pipe polynomial for the first
+// kPolyPairs of every 16 pairs), so an E4M3 code differs only where y lies
+// within a few FP32 ulps of a rounding boundary.
+template <bool kMasked>
+__device__ __forceinline__ void softmax_chunk(const uint32_t (&s)[32], float c, float neg_m, int key0,
+                                              int valid, float2 (&lsum)[4], uint32_t* pk) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 sf = make_float2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+    const float2 sv = fadd2(sf, make_float2(-kSBias, -kSBias));       // exact integer S
+    const float2 t = fmul2(sv, make_float2(c, c));
+    const float2 u = fadd2(t, make_float2(neg_m, neg_m));
+    float2 p;
+    if (i < kPolyPairs) {
+      p = exp2_poly2(u);
+    } else {
+      p.x = ex2_approx(u.x);
+      p.y = ex2_approx(u.y);
+    }
+    float2 y = fmul2(p, make_float2(448.f, 448.f));
+    if (kMasked) {
+      if (key0 + 2 * i >= valid) y.x = 0.f;
+      if (key0 + 2 * i + 1 >= valid) y.y = 0.f;
+    }
+    lsum[i & 3] = fadd2(lsum[i & 3], y);   // four independent partial sums
+    const uint32_t h16 = cvt_e4m3x2(y.x, y.y);
+    if (i & 1)
+      pk[i >> 1] |= h16 << 16;
+    else
+      pk[i >> 1] = h16;
+  }
+}
+
+// Max of one 32-column chunk of biased scores, valid keys only.
+template <bool kMasked>
+__device__ __forceinline__ float chunk_max(const uint32_t (&a)[32], int key0, int valid) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = __uint_as_float(a[i]);
+    if (kMasked && key0 + i >= valid) v[i] = 0.f;   // below every biased score
+  }
+  float w[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  w[10] = fmaxf(v[30], v[31]);
+  const float x0 = fmax3(w[0], w[1], w[2]);
+  const float x1 = fmax3(w[3], w[4], w[5]);
+  const float x2 = fmax3(w[6], w[7], w[8]);
+  return fmaxf(fmax3(x0, x1, x2), fmaxf(w[9], w[10]));
+}
+
+// Row max over all 128 keys of S (biased floats) in TMEM, 32 columns at a
+// time with the next load in flight while the current chunk is reduced.
+template <bool kMasked>
+__device__ __forceinline__ void tmem_row_max(uint32_t taddr, int valid, float c0, float c1, float& tmax) {
+  uint32_t a[32], b[32];
+  float mx0, mx1;
+  tmem_ld32(taddr, a);
+  tmem_wait_ld();
+  reg_fence(a);
+  tmem_ld32(taddr + 32, b);
+  mx0 = chunk_max<kMasked>(a, 0, valid);
+  tmem_wait_ld();
+  reg_fence(b);
+  tmem_ld32(taddr + 64, a);
+  mx0 = fmaxf(mx0, chunk_max<kMasked>(b, 32, valid));
+  tmem_wait_ld();
+  reg_fence(a);
+  tmem_ld32(taddr + 96, b);
+  mx1 = chunk_max<kMasked>(a, 64, valid);
+  tmem_wait_ld();
+  reg_fence(b);
+  mx1 = fmaxf(mx1, chunk_max<kMasked>(b, 96, valid));
+  tmax = __fmul_rn(__fsub_rn(mx0, kSBias), c0);
+  if (!kMasked || valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(mx1, kSBias), c1));
+}
+
+// Exponentials of this thread's 64 keys (keys key0 .. key0+63 at taddr):
+// row-sum and 16 words of E4M3 codes.
+template <bool kMasked>
+__device__ __forceinline__ void tmem_half_exp(uint32_t taddr, float c, float neg_m, int key0, int valid,
+                                              float2 (&lsum)[4], uint32_t* pk) {
+  uint32_t a[32], b[32];
+  tmem_ld32(taddr, a);
+  tmem_wait_ld();
+  reg_fence(a);
+  tmem_ld32(taddr + 32, b);
+  softmax_chunk<kMasked>(a, c, neg_m, key0, valid, lsum, pk);
+  tmem_wait_ld();
+  reg_fence(b);
+  softmax_chunk<kMasked>(b, c, neg_m, key0 + 32, valid, lsum, pk + 8);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
   using L = AttnSmem<D>;
@@ -106,17 +220,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nkv = prm.nkv;
   const int64_t tmo = prm.timeout_ns;
 
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 16; ++i) mbar_init(&bars[i], (i == kBarSEmpty || i == kBarPFull) ? 128u : 1u);
+    for (int i = 0; i < 16; ++i)
+      mbar_init(&bars[i], (i == kBarSEmpty || i == kBarPFull) ? static_cast<uint32_t>(kSoftmaxThreads) : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
   for (int i = tid; i < D; i += kAttnThreads) {
-    s_vf[i] = __fdiv_rn(prm.v_scale[static_cast<int64_t>(bh) * D + i], 448.f);
+    s_vf[i] = prm.v_scale[static_cast<int64_t>(bh) * D + i];
     s_vm[i] = prm.v_mean[static_cast<int64_t>(bh) * D + i];
   }
   tc_fence_before();
@@ -126,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem_s = tmem;
   const uint32_t tmem_o = tmem + 128;
 
-  if (warp == 4) {
+  if (warp == kWarpProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -170,7 +285,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdescQK = make_idesc(2u, 1u, 128u, 128u);          // S32 <- S8 x S8
@@ -188,13 +303,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j < nkv) {
           const int st = j & 1;
           if (!mbar_wait_bounded(&bars[kBarKFull + st], static_cast<uint32_t>(j >> 1) & 1, abort_flag, tmo)) break;
-          if (j >= 1 && !mbar_wait_bounded(&bars[kBarSEmpty], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo))
-            break;
+          // Completion j of S-empty: the softmax warps have re-seeded S with the bias.
+          if (!mbar_wait_bounded(&bars[kBarSEmpty], static_cast<uint32_t>(j) & 1, abort_flag, tmo)) break;
           tc_fence_after();
           const uint64_t kd = st ? kdesc1 : kdesc0;
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(tmem_s, qdesc + 2u * kk, kd + 2u * kk, kIdescQK, kk > 0 ? 1u : 0u);
+            mma_i8_ss(tmem_s, qdesc + 2u * kk, kd + 2u * kk, kIdescQK, 1u);
           tc_commit(&bars[kBarKEmpty + st]);
           tc_commit(&bars[kBarSFull]);
         }
@@ -228,8 +343,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float sl2e = prm.sl2e;
     uint8_t* sP = smem + L::kP;
     float m = -__int_as_float(0x7F800000);
-    float l = 0.f;
+    float l = 0.f;                                // sum of 448 * P~
     bool ok = true;
+    // Seed S with the bias and release it for the first QK^T MMA.
+#pragma unroll
+    for (int cb = 0; cb < kBN; cb += 32) tmem_st32_fill(tmem_s + lane_base + cb, kSBiasBits);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&bars[kBarSEmpty]);
     for (int j = 0; j < nkv; ++j) {
       const float c0 = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
       const float c1 = __fmul_rn(__fmul_rn(qs, ks[2 * j + 1]), sl2e);
@@ -238,52 +359,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sa[32], sb[32], sc[32], sd[32];
-      tmem_ld32(tmem_s + lane_base + 0, sa);
-      tmem_ld32(tmem_s + lane_base + 32, sb);
-      tmem_ld32(tmem_s + lane_base + 64, sc);
-      tmem_ld32(tmem_s + lane_base + 96, sd);
-      tmem_wait_ld();
-      reg_fence(sa);
-      reg_fence(sb);
-      reg_fence(sc);
-      reg_fence(sd);
-      tc_fence_before();
-      mbar_arrive(&bars[kBarSEmpty]);
-
       const int valid = min(kBN, prm.N - j * kBN);
-      int ia = INT_MIN, ib = INT_MIN;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        if (k < valid) ia = max(ia, static_cast<int>(sa[k]));
-        if (k + 32 < valid) ia = max(ia, static_cast<int>(sb[k]));
-        if (k + 64 < valid) ib = max(ib, static_cast<int>(sc[k]));
-        if (k + 96 < valid) ib = max(ib, static_cast<int>(sd[k]));
-      }
-      float tmax = -__int_as_float(0x7F800000);
-      if (valid > 0) tmax = __fmul_rn(__int2float_rn(ia), c0);
-      if (valid > 64) tmax = fmaxf(tmax, __fmul_rn(__int2float_rn(ib), c1));
+      float tmax;
+      if (valid == kBN)
+        tmem_row_max<false>(tmem_s + lane_base, valid, c0, c1, tmax);
+      else
+        tmem_row_max<true>(tmem_s + lane_base, valid, c0, c1, tmax);
       const float m_new = fmaxf(m, tmax);
       const float alpha = ex2_approx(__fsub_rn(m, m_new));
-      const float neg = -m_new;
-      float sum = 0.f;
       uint32_t pk[32];  // 128 E4M3 codes, 4 per word, key order
+      float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+      if (valid == kBN)
+        tmem_half_exp<false>(tmem_s + lane_base, c0, -m_new, 0, valid, lsum, pk);
+      else
+        tmem_half_exp<true>(tmem_s + lane_base, c0, -m_new, 0, valid, lsum, pk);
+      // Ordering point: the first half's codes are complete before the second
+      // half is loaded, so only 64 scores are live at a time.
 #pragma unroll
-      for (int w = 0; w < 32; ++w) {
-        const uint32_t* src = w < 8 ? sa : (w < 16 ? sb : (w < 24 ? sc : sd));
-        const float c = w < 16 ? c0 : c1;
-        float p[4];
+      for (int i = 0; i < 16; ++i) asm volatile("" : "+r"(pk[i])::"memory");
+      if (valid == kBN)
+        tmem_half_exp<false>(tmem_s + lane_base + 64, c1, -m_new, 64, valid, lsum, pk + 16);
+      else
+        tmem_half_exp<true>(tmem_s + lane_base + 64, c1, -m_new, 64, valid, lsum, pk + 16);
+      // Re-seed S with the bias for the next tile's MMA, then release the buffer.
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int key = 4 * w + i;
-          const float pv = ex2_approx(__fmaf_rn(int_to_float(src[(4 * w + i) & 31]), c, neg));
-          p[i] = key < valid ? pv : 0.f;
-          sum = __fadd_rn(sum, p[i]);
-        }
-        pk[w] = cvt_e4m3x2(__fmul_rn(p[0], 448.f), __fmul_rn(p[1], 448.f)) |
-                (cvt_e4m3x2(__fmul_rn(p[2], 448.f), __fmul_rn(p[3], 448.f)) << 16);
-      }
-      l = __fadd_rn(__fmul_rn(l, alpha), sum);
+      for (int cb = 0; cb < kBN; cb += 32) tmem_st32_fill(tmem_s + lane_base + cb, kSBiasBits);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[kBarSEmpty]);
+      const float2 ls2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
+      l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(ls2.x, ls2.y));
 
       if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) {
         ok = false;
@@ -306,7 +412,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_ld();
           reg_fence(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
+          for (int i = 0; i < 32; i += 2) {
+            const float2 r = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                   make_float2(alpha, alpha));
+            o[i] = __float_as_uint(r.x);
+            o[i + 1] = __float_as_uint(r.y);
+          }
           tmem_st32(tmem_o + lane_base + cb, o);
         }
         tmem_wait_st();
@@ -319,6 +430,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (ok && warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(nkv - 1) & 1, abort_flag, tmo)) {
       tc_fence_after();
       const int qrow = qt * kBM + row;
+      // O_acc ~ sum_k P8_k * code_k with P8 ~ 448 P~ and l = sum 448 P~:
+      // O = O_acc * v_scale / l + v_mean.
       const float rl = __fdiv_rn(1.f, l);
       const int64_t obase = ((static_cast<int64_t>(b) * prm.N + qrow) * prm.H + h) * D;
 #pragma unroll
@@ -329,8 +442,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         reg_fence(o);
         float r[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          r[i] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(o[i]), s_vf[cb + i]), rl), s_vm[cb + i]);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 t = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                 make_float2(s_vf[cb + i], s_vf[cb + i + 1]));
+          const float2 u = ffma2(t, make_float2(rl, rl), make_float2(s_vm[cb + i], s_vm[cb + i + 1]));
+          r[i] = u.x;
+          r[i + 1] = u.y;
+        }
         if (qrow < prm.N) {
           if (prm.out_fp32) {
             float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + obase + cb);
@@ -350,7 +468,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       if (prm.lse && qrow < prm.N)
-        prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(l)) * 0.69314718055994531f;
+        prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(l) - kLog2P8) * 0.69314718055994531f;
     }
   }
 
@@ -358,7 +476,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && tid == 0) atomicExch(prm.err, 1);
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -52,6 +52,26 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def attn_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the last ncu capture,
+    if that capture was taken on this workload and on the current kernel source
+    (SHA-256 of the kernel files); None otherwise."""
+    import hashlib
+    pkg = os.path.join(ROOT, "action_diffusion_transformers_b200")
+    try:
+        with open(os.path.join(pkg, "ncu_counters.json")) as f:
+            rec = json.load(f)["sage_attn_kernel<128>"]
+    except (OSError, KeyError, ValueError):
+        return None
+    h = hashlib.sha256()
+    for name in ("sage_attn.cuh", "sage_ptx.cuh"):
+        with open(os.path.join(pkg, "csrc", name), "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -316,7 +336,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "global_batch": w.B * world,
                    "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "sage_attn_kernel<128>",
+                     "frac": achieved / peak, "traffic": attn_traffic(w.name), "kernel": "sage_attn_kernel<128>",
                      "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"},
         "kernels_us": {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
                        "attn": 1e3 * attn_mean_ms},

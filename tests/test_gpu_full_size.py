@@ -1,0 +1,86 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark
+times (the three calls on the whole batch), checked on sampled outputs that
+the oracle computes head by head and row by row:
+
+* quantization codes, scales and means of sampled heads: bit-exact (the
+  oracle runs on those heads' full token columns, so the means are the same);
+* attention output of sampled query rows of sampled heads (FP32 output):
+  max-abs <= 2e-3 and cosine >= 0.9999 against the oracle, and cosine against
+  exact FP64 attention on the BF16 inputs >= 0.999 -- except on the
+  long-video workload, whose Student-t(3) rows make a few softmax rows hinge
+  on large INT8 scores: there the method itself (the oracle, and equally a
+  per-token INT8 variant) reaches about 0.998, so the check is >= 0.997;
+* the BF16 output equals the RNE rounding of the FP32 output on those rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import numerics as nm
+from oracle import sage_oracle as so
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+def _dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _rows(N, seed, count=192):
+    rng = np.random.default_rng(seed)
+    fixed = {0, 1, 63, 64, 127, N - 1, N // 2}
+    last0 = (N // 128) * 128
+    fixed.update(range(last0, N))                       # a ragged last tile, all of it
+    fixed.update(rng.choice(N, size=count, replace=False).tolist())
+    return np.asarray(sorted(r for r in fixed if r < N), dtype=np.int64)
+
+
+def _cos(a, b):
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+
+@pytest.mark.parametrize("name", ["action_dit", "mid_video", "long_video", "ragged"])
+def test_full_size_sampled_parity(adt, name):
+    w = synth.WORKLOADS[name]
+    qb, kb, vb = synth.generate(w)
+    q, k, v = _dev(qb), _dev(kb), _dev(vb)
+    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens)
+    out16 = buf.run(q, k, v)
+    out32 = torch.empty((w.B, w.N, w.H, w.D), dtype=torch.float32, device="cuda")
+    adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
+                      buf.v_mean, buf.shape, 0.0, out32, True)
+    adt.sage_check()
+
+    heads = [(0, 0), (w.B - 1, w.H - 1), (0, w.H // 2)]
+    rows = _rows(w.N, w.seed)
+    for i, (b, h) in enumerate(heads):
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1), slice(None))
+        ref_qk = so.quant_qk(qb[sl], kb[sl])
+        ref_v = so.quant_v(vb[sl])
+        got = lambda t: t[b:b + 1, h:h + 1].cpu().numpy()  # noqa: E731
+        assert np.array_equal(got(buf.q_codes), ref_qk["q_codes"])
+        assert np.array_equal(got(buf.k_codes), ref_qk["k_codes"])
+        assert np.array_equal(got(buf.q_scale).view(np.uint32), ref_qk["q_scale"].view(np.uint32))
+        assert np.array_equal(got(buf.k_scale).view(np.uint32), ref_qk["k_scale"].view(np.uint32))
+        assert np.array_equal(buf.k_mean[b:b + 1, h:h + 1].cpu().view(torch.int16).numpy().view(np.uint16),
+                              ref_qk["k_mean"])
+        assert np.array_equal(got(buf.v_codes_t), ref_v["v_codes_t"])
+        assert np.array_equal(got(buf.v_scale).view(np.uint32), ref_v["v_scale"].view(np.uint32))
+        assert np.array_equal(got(buf.v_mean).view(np.uint32), ref_v["v_mean"].view(np.uint32))
+        if i >= 2:
+            continue
+        ref = so.attn_fwd(ref_qk["q_codes"], ref_qk["q_scale"], ref_qk["k_codes"], ref_qk["k_scale"],
+                          ref_v["v_codes_t"], ref_v["v_scale"], ref_v["v_mean"], w.N, rows=rows)[0, :, 0, :]
+        g32 = out32[b, rows, h, :].cpu().numpy()
+        assert np.all(np.isfinite(g32))
+        err = np.abs(g32 - ref).max()
+        assert err <= 2e-3, f"{name} head {(b, h)}: max-abs {err}"
+        assert _cos(g32, ref) >= 0.9999
+        exact = so.attn_exact_fp64(*(synth.bits_to_f64(x[sl]) for x in (qb, kb, vb)), w.N, rows=rows)[0, :, 0, :]
+        floor = 0.997 if name == "long_video" else 0.999
+        assert _cos(g32, exact) >= floor, f"{name} head {(b, h)}: cos vs exact {_cos(g32, exact)}"
+        g16 = out16[b, rows, h, :].cpu().view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(g16, nm.f32_to_bf16_bits(g32))
