@@ -281,11 +281,11 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  const dim3 g(Npad / sage::kQKBlock, s.H, 2 * s.B);
+  const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
   if (s.D == 128)
-    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
   else
-    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
   return launch_check("sage_quant_qk launch");
 }
 
@@ -459,11 +459,11 @@ sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  const dim3 g(Npad / sage::kQKBlock, s.H, 2 * s.B);
+  const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
   if (s.D == 128)
-    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
   else
-    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
   return launch_check("sage_quant_qk_static launch");
 }
 

@@ -56,44 +56,39 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
   const int n1 = min(N, n0 + kSumBlock);
   const uint16_t* p = x + (static_cast<int64_t>(b) * N + n0) * tok_stride + ch0;
   double s[8];
-  float mn[8], mx[8];
+  // min / max kept as packed BF16 pairs (exact: the inputs are BF16)
+  __nv_bfloat162 mn[4], mx[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s[i] = 0.0;
-    mn[i] = __int_as_float(0x7F800000);
-    mx[i] = -__int_as_float(0x7F800000);
+  for (int i = 0; i < 8; ++i) s[i] = 0.0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mn[i] = __floats2bfloat162_rn(__int_as_float(0x7F800000), __int_as_float(0x7F800000));
+    mx[i] = __floats2bfloat162_rn(-__int_as_float(0x7F800000), -__int_as_float(0x7F800000));
   }
+  auto accumulate = [&](const uint4& raw) {
+    float f[8];
+    unpack8(raw, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i] = __dadd_rn(s[i], static_cast<double>(f[i]));
+    if (kMinMax) {
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        mn[i] = __hmin2(mn[i], v);
+        mx[i] = __hmax2(mx[i], v);
+      }
+    }
+  };
   int n = n0;
   for (; n + 8 <= n1; n += 8) {
     uint4 raw[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) raw[t] = ld_nc_16(p + static_cast<int64_t>(n - n0 + t) * tok_stride);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      float f[8];
-      unpack8(raw[t], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        s[i] = __dadd_rn(s[i], static_cast<double>(f[i]));
-        if (kMinMax) {
-          mn[i] = fminf(mn[i], f[i]);
-          mx[i] = fmaxf(mx[i], f[i]);
-        }
-      }
-    }
+    for (int t = 0; t < 8; ++t) accumulate(raw[t]);
   }
-  for (; n < n1; ++n) {
-    float f[8];
-    unpack8(ld_nc_16(p + static_cast<int64_t>(n - n0) * tok_stride), f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      s[i] = __dadd_rn(s[i], static_cast<double>(f[i]));
-      if (kMinMax) {
-        mn[i] = fminf(mn[i], f[i]);
-        mx[i] = fmaxf(mx[i], f[i]);
-      }
-    }
-  }
+  for (; n < n1; ++n) accumulate(ld_nc_16(p + static_cast<int64_t>(n - n0) * tok_stride));
   const int64_t o = (static_cast<int64_t>(b) * nsb + c) * HD + ch0;
   double2* ps = reinterpret_cast<double2*>(psum + o);
 #pragma unroll
@@ -101,10 +96,10 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
   if (kMinMax) {
     float4* pn = reinterpret_cast<float4*>(pmin + o);
     float4* px = reinterpret_cast<float4*>(pmax + o);
-    pn[0] = make_float4(mn[0], mn[1], mn[2], mn[3]);
-    pn[1] = make_float4(mn[4], mn[5], mn[6], mn[7]);
-    px[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
-    px[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
+    pn[0] = make_float4(__low2float(mn[0]), __high2float(mn[0]), __low2float(mn[1]), __high2float(mn[1]));
+    pn[1] = make_float4(__low2float(mn[2]), __high2float(mn[2]), __low2float(mn[3]), __high2float(mn[3]));
+    px[0] = make_float4(__low2float(mx[0]), __high2float(mx[0]), __low2float(mx[1]), __high2float(mx[1]));
+    px[1] = make_float4(__low2float(mx[2]), __high2float(mx[2]), __low2float(mx[3]), __high2float(mx[3]));
   }
 }
 
@@ -216,26 +211,38 @@ __global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restric
 }
 
 // ----------------------------------------------------------------------------
-// INT8 block quantization.  CTA = one (b, h, 64-token block) of Q (z even) or
-// K (z odd, centred by mean_k and rounded to BF16 first).  256 threads: D/8
-// threads cover one token row (8 channels each), 256/(D/8) rows per pass.
-// Grid (Npad/64, H, 2*B).
+// INT8 block quantization.  CTA = one (b, h, 128-token tile = two 64-token
+// scale blocks) of K (z < B: centred by mean_k and rounded to BF16 first) or Q
+// (z >= B).  K runs first so that its second read follows the column-sum pass
+// while K is still in L2.  256 threads: D/8 threads cover one token row (8
+// channels each); each thread holds 128 / (256 / (D/8)) tokens, so 8 16-byte
+// loads are in flight per thread at D = 128.  Grid (Npad/128, H, 2*B).
+// Rounding: RNE(RN(x * inv)) is formed by adding 1.5 * 2^23 (exact here:
+// |x * inv| <= 127 * (1 + 2^-23)), which keeps the conversion on the FMA pipe.
 // ----------------------------------------------------------------------------
+__device__ __forceinline__ int rne_small(float y) {
+  return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict__ q,
-                                                      const uint16_t* __restrict__ k, int N, int H, int Npad,
-                                                      int64_t tok_stride, const uint16_t* __restrict__ k_mean,
+                                                      const uint16_t* __restrict__ k, int N, int B, int H,
+                                                      int Npad, int64_t tok_stride,
+                                                      const uint16_t* __restrict__ k_mean,
                                                       int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
                                                       int8_t* __restrict__ k_codes,
                                                       float* __restrict__ k_scale) {
   constexpr int kLPR = D / 8;             // threads per token row
   constexpr int kRPP = 256 / kLPR;        // token rows per pass
-  constexpr int kTPT = kQKBlock / kRPP;   // tokens per thread
-  __shared__ float red[8];
-  const int blk = blockIdx.x;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z >> 1;
-  const bool is_k = blockIdx.z & 1;
+  constexpr int kTPT = kTile / kRPP;      // tokens per thread (half in each 64-token block)
+  constexpr int kHalf = kTPT / 2;
+  __shared__ float red[8][2];
+  const int tile = blockIdx.x;
+  const bool is_k = static_cast<int>(blockIdx.z) < B;
+  // K heads are visited last-to-first: the column-sum pass just streamed K in
+  // head order, so the most recently read heads (still in L2) come first.
+  const int h = is_k ? H - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
+  const int b = is_k ? blockIdx.z : blockIdx.z - B;
   const uint16_t* src = is_k ? k : q;
   const int cg = threadIdx.x % kLPR;
   const int r0 = threadIdx.x / kLPR;
@@ -246,52 +253,72 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
     const uint4 mraw = *reinterpret_cast<const uint4*>(k_mean + (static_cast<int64_t>(b) * H + h) * D + d0);
     unpack8(mraw, mean);
   }
-  float x[kTPT][8];
-  float amax = 0.f;
+  uint4 raw[kTPT];
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
-    const int n = blk * kQKBlock + r0 + t * kRPP;
-    if (n < N) {
-      const uint4 raw = ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0);
-      unpack8(raw, x[t]);
-      if (is_k) {
+    const int n = tile * kTile + r0 + t * kRPP;
+    raw[t] = n < N ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
+                   : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float x[kTPT][8];
+  float amax[2] = {0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[t][i] = bf16_bits_to_float(float_to_bf16_bits(__fsub_rn(x[t][i], mean[i])));
-      }
-    } else {
+  for (int t = 0; t < kTPT; ++t) {
+    const int n = tile * kTile + r0 + t * kRPP;
+    unpack8(raw[t], x[t]);
+    if (is_k) {
+      if (n < N) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[t][i] = 0.f;
+        for (int i = 0; i < 8; i += 2) {
+          const __nv_bfloat162 c2 =
+              __floats2bfloat162_rn(__fsub_rn(x[t][i], mean[i]), __fsub_rn(x[t][i + 1], mean[i + 1]));
+          x[t][i] = __low2float(c2);
+          x[t][i + 1] = __high2float(c2);
+        }
+      }  // padded rows stay 0
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[t][i]));
+    for (int i = 0; i < 8; ++i) amax[t / kHalf] = fmaxf(amax[t / kHalf], fabsf(x[t][i]));
   }
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  for (int o = 16; o >= 1; o >>= 1) {
+    amax[0] = fmaxf(amax[0], __shfl_xor_sync(0xFFFFFFFFu, amax[0], o));
+    amax[1] = fmaxf(amax[1], __shfl_xor_sync(0xFFFFFFFFu, amax[1], o));
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[threadIdx.x >> 5][0] = amax[0];
+    red[threadIdx.x >> 5][1] = amax[1];
+  }
   __syncthreads();
-  amax = red[0];
+  float scale[2], inv[2];
 #pragma unroll
-  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
-  float scale = 0.f, inv = 0.f;
-  if (amax > 0.f) {
-    scale = __fdiv_rn(amax, 127.f);
-    inv = __fdiv_rn(127.f, amax);
+  for (int blk = 0; blk < 2; ++blk) {
+    float a = red[0][blk];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][blk]);
+    scale[blk] = 0.f;
+    inv[blk] = 0.f;
+    if (a > 0.f) {
+      scale[blk] = __fdiv_rn(a, 127.f);
+      inv[blk] = __fdiv_rn(127.f, a);
+    }
   }
   const int64_t bh = static_cast<int64_t>(b) * H + h;
   int8_t* dst = is_k ? k_codes : q_codes;
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
-    const int n = blk * kQKBlock + r0 + t * kRPP;
+    const int n = tile * kTile + r0 + t * kRPP;
+    const float iv = inv[t / kHalf];
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      int c = __float2int_rn(__fmul_rn(x[t][i], inv));
+      int c = rne_small(__fmul_rn(x[t][i], iv));
       c = max(-127, min(127, c));
       w[i >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (i & 3));
     }
     *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w[0], w[1]);
   }
-  if (threadIdx.x == 0) (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + blk] = scale;
+  if (threadIdx.x < 2) (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + tile * 2 + threadIdx.x] = scale[threadIdx.x];
 }
 
 // ----------------------------------------------------------------------------
@@ -311,7 +338,8 @@ __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v,
   constexpr int kPitch = D + 16;          // bytes per token row of the shared tile
   __shared__ __align__(16) uint8_t tile[kTile * kPitch];
   const int n0 = blockIdx.x * kTile;
-  const int h = blockIdx.y;
+  // Heads last-to-first: the statistics pass just streamed V in head order.
+  const int h = H - 1 - static_cast<int>(blockIdx.y);
   const int b = blockIdx.z;
   const int cg = threadIdx.x % kLPR;
   const int r0 = threadIdx.x / kLPR;
@@ -340,19 +368,34 @@ __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v,
     *reinterpret_cast<uint2*>(tile + nl * kPitch + d0) = make_uint2(w0, w1);
   }
   __syncthreads();
-  constexpr int kChunks = D * (kTile / 16);  // 16-token pieces of all channel rows
-  for (int idx = threadIdx.x; idx < kChunks; idx += 256) {
-    const int d = idx % D;
-    const int qc = idx / D;
-    uint32_t w[4];
+  // Phase 2: a thread owns 4 channels x 16 tokens.  It reads 16 words (4
+  // channels of one token each), transposes each 4x4 byte block with prmt, and
+  // writes 4 transposed 16-byte pieces (16 tokens of one channel each).
+  constexpr int kUnits = (D / 4) * (kTile / 16);
+  for (int u = threadIdx.x; u < kUnits; u += 256) {
+    const int d4 = u % (D / 4);
+    const int qc = u / (D / 4);
+    uint32_t col[4][4];  // col[c][j]: channel 4*d4+c, tokens qc*16 + 4j .. +3
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      uint32_t acc = 0u;
+      uint32_t r[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc |= static_cast<uint32_t>(tile[(qc * 16 + j * 4 + i) * kPitch + d]) << (8 * i);
-      w[j] = acc;
+      for (int i = 0; i < 4; ++i)
+        r[i] = *reinterpret_cast<const uint32_t*>(tile + (qc * 16 + 4 * j + i) * kPitch + 4 * d4);
+      // r[i] holds channels 0..3 of token i; gather byte c of every token.
+      const uint32_t lo01 = __byte_perm(r[0], r[1], 0x5140);   // t0c0 t1c0 t0c1 t1c1
+      const uint32_t lo23 = __byte_perm(r[2], r[3], 0x5140);   // t2c0 t3c0 t2c1 t3c1
+      const uint32_t hi01 = __byte_perm(r[0], r[1], 0x7362);   // t0c2 t1c2 t0c3 t1c3
+      const uint32_t hi23 = __byte_perm(r[2], r[3], 0x7362);   // t2c2 t3c2 t2c3 t3c3
+      col[0][j] = __byte_perm(lo01, lo23, 0x5410);
+      col[1][j] = __byte_perm(lo01, lo23, 0x7632);
+      col[2][j] = __byte_perm(hi01, hi23, 0x5410);
+      col[3][j] = __byte_perm(hi01, hi23, 0x7632);
     }
-    *reinterpret_cast<uint4*>(out + (bhd + d) * Npad + n0 + qc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4*>(out + (bhd + 4 * d4 + c) * Npad + n0 + qc * 16) =
+          make_uint4(col[c][0], col[c][1], col[c][2], col[c][3]);
   }
 }
 
