@@ -1,20 +1,24 @@
 // sage_attn.cuh - quantized attention forward on sm_100a tensor cores.
 //
 // One CTA computes one 128-row query tile of one (b, h).  Warp roles:
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Per tile it
-//              reads S from TMEM twice (row max, then exponentials 64 keys at a
-//              time, so only 64 scores are ever live in registers), writes P as
-//              E4M3 into a 128B-swizzled shared tile, rescales the O
-//              accumulator in TMEM when its row max moves, and runs the
-//              epilogue.  Two CTAs share an SM; their softmax warps are
-//              independent, so their MUFU-heavy and ALU-heavy phases interleave.
+//   warps 0-7  softmax: two threads per query row.  Warp w reads TMEM lane
+//              quadrant w % 4 (query rows 32 (w % 4) ..) and score columns
+//              64 (w / 4) .. + 63, i.e. one 64-key scale block.  Per tile a
+//              thread loads its 64 scores once, reduces their max, swaps it
+//              with its partner thread through shared memory (an mbarrier per
+//              warp pair, so the wait is bounded), then forms E4M3 codes of
+//              P~ * 448 for its 64 keys, writes them into a 128B-swizzled
+//              shared P tile, rescales its half of the O accumulator in TMEM
+//              when the row max moves, and runs its half of the epilogue.
+//              Two CTAs share an SM, so 16 softmax warps hide each other's
+//              latencies.
 // S is accumulated onto the integer 0x4B400000 (the bits of 1.5 * 2^23) that
 // the softmax warps write into the S columns before each QK^T MMA: read as a
 // float, a loaded S word is then exactly 1.5 * 2^23 + S (|S| <= 127^2 * D <
 // 2^22), so one exact subtraction converts it, two at a time with f32x2.
-//   warp 4     producer: one thread issues TMA tile loads (Q once; K and V
+//   warp 8     producer: one thread issues TMA tile loads (Q once; K and V
 //              tiles into 2-stage rings).
-//   warp 5     MMA: allocates TMEM; one thread issues
+//   warp 9     MMA: allocates TMEM; one thread issues
 //              S  = Qc Kc^T  tcgen05.mma kind::i8      (INT32 accumulate)
 //              O += P8 V8    tcgen05.mma kind::f8f6f4  (FP32 accumulate).
 // TMEM (256 columns): S at columns [0, 128), O at [128, 128 + D).
@@ -38,18 +42,15 @@ namespace sage {
 
 constexpr int kBM = 128;   // query rows per tile
 constexpr int kBN = 128;   // keys per tile
-constexpr int kAttnThreads = 192;      // 4 softmax warps + producer + MMA
-constexpr int kSoftmaxThreads = 128;   // one thread per query row
-constexpr int kWarpProducer = 4;
-constexpr int kWarpMma = 5;
+constexpr int kAttnThreads = 320;      // 8 softmax warps + producer + MMA
+constexpr int kSoftmaxThreads = 256;   // two threads per query row
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kNumBars = 18;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSBiasBits = 0x4B400000u;   // S accumulates onto these bits
 constexpr float kSBias = 12582912.0f;          // their float value, 1.5 * 2^23
-constexpr float kLog2P8 = 8.8073549220576041f; // log2(448): the row sum holds 448 * P~
-#ifndef SAGE_POLY_PAIRS
-#define SAGE_POLY_PAIRS 0                      // of every 16 column pairs, exp2 on the FMA pipe
-#endif
-constexpr int kPolyPairs = SAGE_POLY_PAIRS;
+constexpr float kLog2P8 = 8.8073549220576041f; // log2(448): the P scale, folded into the exponent
 
 template <int D>
 struct AttnSmem {
@@ -65,8 +66,9 @@ struct AttnSmem {
   static constexpr int kP = kV1 + kVBytes;
   static constexpr int kVf = kP + kPBytes;     // D floats: v_scale
   static constexpr int kVm = kVf + 4 * D;      // D floats: v_mean
-  static constexpr int kBar = kVm + 4 * D;     // 16 mbarriers
-  static constexpr int kMisc = kBar + 16 * 8;  // tmem slot, abort flag
+  static constexpr int kX = kVm + 4 * D;       // [2 phases][2 halves][128 rows] floats: row max / sum swap
+  static constexpr int kBar = kX + 2 * 2 * kBM * 4;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024; // slack for 1024-byte alignment
 };
@@ -86,7 +88,8 @@ struct AttnParams {
 };
 
 enum : int { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-             kBarSEmpty = 10, kBarPFull = 11, kBarPVDone = 12, kBarDrain = 13 };
+             kBarSEmpty = 10, kBarPFull = 11, kBarPVDone = 12, kBarDrain = 13,
+             kBarPair = 14 /* 4: one per warp pair sharing a lane quadrant */ };
 
 // Bounded wait whose outcome is the same in every lane of the warp, so that a
 // warp never splits in front of a warp-collective tcgen05 instruction.
@@ -100,101 +103,69 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
   return __int2float_rn(static_cast<int>(s));
 }
 
-// One 32-column chunk of a score row, with the contract's rounding steps:
-// t = RN(S * c), u = RN(t - m_new), p = 2^u, y = RN(p * 448) -> E4M3 code;
-// the row sum accumulates y (= 448 * P~).  Only the exp2 itself differs from
-// the contract (hardware ex2.approx, or the FMA-pipe polynomial for the first
-// kPolyPairs of every 16 pairs), so an E4M3 code differs only where y lies
-// within a few FP32 ulps of a rounding boundary.
-template <bool kMasked>
-__device__ __forceinline__ void softmax_chunk(const uint32_t (&s)[32], float c, float neg_m, int key0,
-                                              int valid, float2 (&lsum)[4], uint32_t* pk) {
+// The contract's exponentials for 32 of this thread's keys (16 pairs of biased
+// scores s; valid counts from the first of them): u = RN(S * c + e) with e = RN(log2 448 - m_new) (one fused
+// multiply-add), y = exp2_fixed(u) = P~ * 448 -> E4M3 code; the row sum
+// accumulates y.  Every step is a binary32 operation with fixed rounding, so y
+// and its code equal the oracle's bit for bit.  kClamp: some u of this warp's
+// tile may be below -126.  pk[w] holds the codes of keys 4w .. 4w+3.
+template <bool kMasked, bool kClamp>
+__device__ __forceinline__ void softmax_quarter(const f32x2_t (&s)[16], f32x2_t c2, f32x2_t e2, int valid,
+                                                const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
+  f32x2_t prev = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float2 sf = make_float2(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
-    const float2 sv = fadd2(sf, make_float2(-kSBias, -kSBias));       // exact integer S
-    const float2 t = fmul2(sv, make_float2(c, c));
-    const float2 u = fadd2(t, make_float2(neg_m, neg_m));
-    float2 p;
-    if (i < kPolyPairs) {
-      p = exp2_poly2(u);
-    } else {
-      p.x = ex2_approx(u.x);
-      p.y = ex2_approx(u.y);
+    const f32x2_t sv = x2_sub(s[i], k.round);            // exact integer S (the S bias is 1.5 * 2^23 too)
+    f32x2_t u = x2_fma(sv, c2, e2);
+    if (kClamp) {
+      const float lo = fmaxf(x2_lo(u), kExp2Min);
+      const float hi = fmaxf(x2_hi(u), kExp2Min);
+      u = (static_cast<f32x2_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
     }
-    float2 y = fmul2(p, make_float2(448.f, 448.f));
+    f32x2_t y = exp2_fixed_x2(u, k);
     if (kMasked) {
-      if (key0 + 2 * i >= valid) y.x = 0.f;
-      if (key0 + 2 * i + 1 >= valid) y.y = 0.f;
+      const uint32_t lo = 2 * i < valid ? static_cast<uint32_t>(y) : 0u;
+      const uint32_t hi = 2 * i + 1 < valid ? static_cast<uint32_t>(y >> 32) : 0u;
+      y = (static_cast<f32x2_t>(hi) << 32) | lo;
     }
-    lsum[i & 3] = fadd2(lsum[i & 3], y);   // four independent partial sums
-    const uint32_t h16 = cvt_e4m3x2(y.x, y.y);
+    lsum[i & 3] = x2_add(lsum[i & 3], y);              // four independent partial sums
     if (i & 1)
-      pk[i >> 1] |= h16 << 16;
+      pk[i >> 1] = x2_e4m3x4(prev, y);
     else
-      pk[i >> 1] = h16;
+      prev = y;
   }
 }
 
-// Max of one 32-column chunk of biased scores, valid keys only.
+// Max over the valid keys and min over all keys of this thread's 64 biased scores.
 template <bool kMasked>
-__device__ __forceinline__ float chunk_max(const uint32_t (&a)[32], int key0, int valid) {
-  float v[32];
+__device__ __forceinline__ void half_minmax(const f32x2_t (&s)[32], int valid, float& mx, float& mn) {
+  float v[64];
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    v[i] = __uint_as_float(a[i]);
-    if (kMasked && key0 + i >= valid) v[i] = 0.f;   // below every biased score
+    v[2 * i] = x2_lo(s[i]);
+    v[2 * i + 1] = x2_hi(s[i]);
   }
-  float w[11];
+  float w[22];
 #pragma unroll
-  for (int i = 0; i < 10; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  w[10] = fmaxf(v[30], v[31]);
-  const float x0 = fmax3(w[0], w[1], w[2]);
-  const float x1 = fmax3(w[3], w[4], w[5]);
-  const float x2 = fmax3(w[6], w[7], w[8]);
-  return fmaxf(fmax3(x0, x1, x2), fmaxf(w[9], w[10]));
-}
-
-// Row max over all 128 keys of S (biased floats) in TMEM, 32 columns at a
-// time with the next load in flight while the current chunk is reduced.
-template <bool kMasked>
-__device__ __forceinline__ void tmem_row_max(uint32_t taddr, int valid, float c0, float c1, float& tmax) {
-  uint32_t a[32], b[32];
-  float mx0, mx1;
-  tmem_ld32(taddr, a);
-  tmem_wait_ld();
-  reg_fence(a);
-  tmem_ld32(taddr + 32, b);
-  mx0 = chunk_max<kMasked>(a, 0, valid);
-  tmem_wait_ld();
-  reg_fence(b);
-  tmem_ld32(taddr + 64, a);
-  mx0 = fmaxf(mx0, chunk_max<kMasked>(b, 32, valid));
-  tmem_wait_ld();
-  reg_fence(a);
-  tmem_ld32(taddr + 96, b);
-  mx1 = chunk_max<kMasked>(a, 64, valid);
-  tmem_wait_ld();
-  reg_fence(b);
-  mx1 = fmaxf(mx1, chunk_max<kMasked>(b, 96, valid));
-  tmax = __fmul_rn(__fsub_rn(mx0, kSBias), c0);
-  if (!kMasked || valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(mx1, kSBias), c1));
-}
-
-// Exponentials of this thread's 64 keys (keys key0 .. key0+63 at taddr):
-// row-sum and 16 words of E4M3 codes.
-template <bool kMasked>
-__device__ __forceinline__ void tmem_half_exp(uint32_t taddr, float c, float neg_m, int key0, int valid,
-                                              float2 (&lsum)[4], uint32_t* pk) {
-  uint32_t a[32], b[32];
-  tmem_ld32(taddr, a);
-  tmem_wait_ld();
-  reg_fence(a);
-  tmem_ld32(taddr + 32, b);
-  softmax_chunk<kMasked>(a, c, neg_m, key0, valid, lsum, pk);
-  tmem_wait_ld();
-  reg_fence(b);
-  softmax_chunk<kMasked>(b, c, neg_m, key0 + 32, valid, lsum, pk + 8);
+  for (int i = 0; i < 21; ++i) w[i] = fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  w[21] = v[63];
+  float x[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) x[i] = fmin3(w[3 * i], w[3 * i + 1], w[3 * i + 2]);
+  x[7] = w[21];
+  mn = fminf(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], fminf(x[5], fminf(x[6], x[7]))));
+  if (kMasked) {
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (i >= valid) v[i] = 0.f;                        // below every biased score
+  }
+#pragma unroll
+  for (int i = 0; i < 21; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  w[21] = v[63];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) x[i] = fmax3(w[3 * i], w[3 * i + 1], w[3 * i + 2]);
+  x[7] = w[21];
+  mx = fmaxf(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], fmaxf(x[5], fmaxf(x[6], x[7]))));
 }
 
 template <int D>
@@ -225,8 +196,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 16; ++i)
-      mbar_init(&bars[i], (i == kBarSEmpty || i == kBarPFull) ? static_cast<uint32_t>(kSoftmaxThreads) : 1u);
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1u;
+      if (i == kBarSEmpty || i == kBarPFull) count = kSoftmaxThreads;
+      if (i >= kBarPair) count = 64u;
+      mbar_init(&bars[i], count);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -335,90 +310,113 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int row = tid;                          // TMEM lane == query row in tile
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int quad = warp & 3;                    // TMEM lane quadrant
+    const int half = warp >> 2;                   // score columns 64 half .. + 63
+    const int row = quad * 32 + lane;             // TMEM lane == query row in tile
+    constexpr int kOH = D / 2;                    // O / output columns per thread
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t ts = tmem_s + lane_base + static_cast<uint32_t>(half * 64);
+    const uint32_t to = tmem_o + lane_base + static_cast<uint32_t>(half * kOH);
+    uint64_t* pair_bar = &bars[kBarPair + quad];
+    float* xch = reinterpret_cast<float*>(smem + L::kX);   // [phase & 1][half][row]
     const int nqb = prm.Npad / 64;
     const float qs = prm.q_scale[static_cast<int64_t>(bh) * nqb + qt * 2 + (row >> 6)];
-    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * nqb;
+    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * nqb + half;  // this half's key block
     const float sl2e = prm.sl2e;
     uint8_t* sP = smem + L::kP;
-    float m = -__int_as_float(0x7F800000);
-    float l = 0.f;                                // sum of 448 * P~
+    const float kNegInf = -__int_as_float(0x7F800000);
+    float m = kNegInf;
+    float l = 0.f;                                // this half's sum of P~ * 448
     bool ok = true;
-    // Seed S with the bias and release it for the first QK^T MMA.
-#pragma unroll
-    for (int cb = 0; cb < kBN; cb += 32) tmem_st32_fill(tmem_s + lane_base + cb, kSBiasBits);
+    const Exp2Consts ek;
+    static_assert(kSBias == kExp2Round, "the S bias doubles as the exp2 rounding constant");
+    // Seed this thread's S columns with the bias and release them for the first QK^T MMA.
+    tmem_st32_fill(ts, kSBiasBits);
+    tmem_st32_fill(ts + 32, kSBiasBits);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&bars[kBarSEmpty]);
     for (int j = 0; j < nkv; ++j) {
-      const float c0 = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
-      const float c1 = __fmul_rn(__fmul_rn(qs, ks[2 * j + 1]), sl2e);
+      const float c = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
       if (!warp_wait(&bars[kBarSFull], static_cast<uint32_t>(j) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int valid = min(kBN, prm.N - j * kBN);
-      float tmax;
-      if (valid == kBN)
-        tmem_row_max<false>(tmem_s + lane_base, valid, c0, c1, tmax);
-      else
-        tmem_row_max<true>(tmem_s + lane_base, valid, c0, c1, tmax);
-      const float m_new = fmaxf(m, tmax);
-      const float alpha = ex2_approx(__fsub_rn(m, m_new));
-      uint32_t pk[32];  // 128 E4M3 codes, 4 per word, key order
-      float2 lsum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-      if (valid == kBN)
-        tmem_half_exp<false>(tmem_s + lane_base, c0, -m_new, 0, valid, lsum, pk);
-      else
-        tmem_half_exp<true>(tmem_s + lane_base, c0, -m_new, 0, valid, lsum, pk);
-      // Ordering point: the first half's codes are complete before the second
-      // half is loaded, so only 64 scores are live at a time.
+      const int valid = min(kBN, prm.N - j * kBN) - half * 64;   // valid keys among this thread's 64
+      f32x2_t sp[32];                             // this thread's 64 biased scores
+      tmem_ld64_pairs(ts, sp);
+      // This half's max of t = RN(S * c) (c > 0, so it is the max S scaled), -inf if
+      // no key; and its min S, which bounds every u from below.
+      float th, smin;
+      {
+        float mx, mn;
+        if (valid >= 64)
+          half_minmax<false>(sp, 64, mx, mn);
+        else
+          half_minmax<true>(sp, valid, mx, mn);
+        th = __fmul_rn(__fsub_rn(mx, kSBias), c);
+        if (valid <= 0) th = kNegInf;
+        smin = __fsub_rn(mn, kSBias);
+      }
+      float* xp = xch + (j & 1) * (2 * kBM);
+      xp[half * kBM + row] = th;
+      mbar_arrive(pair_bar);
+      if (!warp_wait(pair_bar, static_cast<uint32_t>(j) & 1, abort_flag, tmo)) {
+        ok = false;
+        break;
+      }
+      const float m_new = fmaxf(m, fmaxf(th, xp[(half ^ 1) * kBM + row]));
+      const float alpha = exp2_fixed(__fsub_rn(m, m_new));
+      const float e = __fsub_rn(kLog2P8, m_new);
+      // u is monotone in S (c > 0), so the smallest u is the min S's; clamping is
+      // the identity unless it is below -126.
+      const bool clamp = __any_sync(0xFFFFFFFFu, __fmaf_rn(smin, c, e) < kExp2Min);
+      uint32_t pk[16];  // this thread's 64 E4M3 codes, 4 per word, key order
+      f32x2_t lsum[4] = {0, 0, 0, 0};
+      const f32x2_t c2 = x2_splat(c);
+      const f32x2_t e2 = x2_splat(e);
+      // Scores again, 32 at a time, so that only 32 are live with the exp2 state.
 #pragma unroll
-      for (int i = 0; i < 16; ++i) asm volatile("" : "+r"(pk[i])::"memory");
-      if (valid == kBN)
-        tmem_half_exp<false>(tmem_s + lane_base + 64, c1, -m_new, 64, valid, lsum, pk + 16);
-      else
-        tmem_half_exp<true>(tmem_s + lane_base + 64, c1, -m_new, 64, valid, lsum, pk + 16);
+      for (int qq = 0; qq < 2; ++qq) {
+        f32x2_t sq[16];
+        tmem_ld32_pairs(ts + 32 * qq, sq);
+        if (valid >= 64 && !clamp)
+          softmax_quarter<false, false>(sq, c2, e2, 64, ek, lsum, pk + 8 * qq);
+        else
+          softmax_quarter<true, true>(sq, c2, e2, valid - 32 * qq, ek, lsum, pk + 8 * qq);
+      }
       // Re-seed S with the bias for the next tile's MMA, then release the buffer.
-#pragma unroll
-      for (int cb = 0; cb < kBN; cb += 32) tmem_st32_fill(tmem_s + lane_base + cb, kSBiasBits);
+      tmem_st32_fill(ts, kSBiasBits);
+      tmem_st32_fill(ts + 32, kSBiasBits);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[kBarSEmpty]);
-      const float2 ls2 = fadd2(fadd2(lsum[0], lsum[1]), fadd2(lsum[2], lsum[3]));
-      l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(ls2.x, ls2.y));
+      const f32x2_t ls2 = x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
+      l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(x2_lo(ls2), x2_hi(ls2)));
 
       if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
-      // P row -> shared tile, 128B swizzle: 16-byte chunk c of row r lives at c ^ (r & 7).
+      // P row -> shared tile, 128B swizzle: 16-byte chunk q of row r lives at q ^ (r & 7).
       uint8_t* prow = sP + row * 128;
 #pragma unroll
-      for (int cch = 0; cch < 8; ++cch) {
-        const int pc = cch ^ (row & 7);
+      for (int cc = 0; cc < 4; ++cc) {
+        const int pc = (half * 4 + cc) ^ (row & 7);
         *reinterpret_cast<uint4*>(prow + pc * 16) =
-            make_uint4(pk[4 * cch], pk[4 * cch + 1], pk[4 * cch + 2], pk[4 * cch + 3]);
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       }
       if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
         tc_fence_after();
+        const f32x2_t a2 = x2_splat(alpha);
 #pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(tmem_o + lane_base + cb, o);
-          tmem_wait_ld();
-          reg_fence(o);
+        for (int cb = 0; cb < kOH; cb += 32) {
+          f32x2_t o[16];
+          tmem_ld32_pairs(to + cb, o);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 r = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
-                                   make_float2(alpha, alpha));
-            o[i] = __float_as_uint(r.x);
-            o[i + 1] = __float_as_uint(r.y);
-          }
-          tmem_st32(tmem_o + lane_base + cb, o);
+          for (int i = 0; i < 16; ++i) o[i] = x2_mul(o[i], a2);
+          tmem_st32_pairs(to + cb, o);
         }
         tmem_wait_st();
       }
@@ -428,47 +426,56 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       m = m_new;
     }
     if (ok && warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(nkv - 1) & 1, abort_flag, tmo)) {
-      tc_fence_after();
-      const int qrow = qt * kBM + row;
-      // O_acc ~ sum_k P8_k * code_k with P8 ~ 448 P~ and l = sum 448 P~:
-      // O = O_acc * v_scale / l + v_mean.
-      const float rl = __fdiv_rn(1.f, l);
-      const int64_t obase = ((static_cast<int64_t>(b) * prm.N + qrow) * prm.H + h) * D;
+      // Row sum: the two halves' sums, added in a fixed order by both threads.
+      float* xp = xch + (nkv & 1) * (2 * kBM);
+      xp[half * kBM + row] = l;
+      mbar_arrive(pair_bar);
+      if (warp_wait(pair_bar, static_cast<uint32_t>(nkv) & 1, abort_flag, tmo)) {
+        const float lt = __fadd_rn(xp[row], xp[kBM + row]);
+        tc_fence_after();
+        const int qrow = qt * kBM + row;
+        // O_acc ~ sum_k P8_k * code_k with P8 ~ 448 P~ and lt = sum 448 P~:
+        // O = RN(O_acc * v_scale) * RN(1 / lt) + v_mean (one fused multiply-add).
+        const float rl = __fdiv_rn(1.f, lt);
+        const int64_t obase = ((static_cast<int64_t>(b) * prm.N + qrow) * prm.H + h) * D + half * kOH;
+        const float* vf = s_vf + half * kOH;
+        const float* vm = s_vm + half * kOH;
 #pragma unroll
-      for (int cb = 0; cb < D; cb += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem_o + lane_base + cb, o);
-        tmem_wait_ld();
-        reg_fence(o);
-        float r[32];
+        for (int cb = 0; cb < kOH; cb += 32) {
+          uint32_t o[32];
+          tmem_ld32(to + cb, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          float r[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float2 t = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
-                                 make_float2(s_vf[cb + i], s_vf[cb + i + 1]));
-          const float2 u = ffma2(t, make_float2(rl, rl), make_float2(s_vm[cb + i], s_vm[cb + i + 1]));
-          r[i] = u.x;
-          r[i + 1] = u.y;
-        }
-        if (qrow < prm.N) {
-          if (prm.out_fp32) {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + obase + cb);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 t = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                   make_float2(vf[cb + i], vf[cb + i + 1]));
+            const float2 u = ffma2(t, make_float2(rl, rl), make_float2(vm[cb + i], vm[cb + i + 1]));
+            r[i] = u.x;
+            r[i + 1] = u.y;
+          }
+          if (qrow < prm.N) {
+            if (prm.out_fp32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + obase + cb);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(prm.out) + obase + cb);
+              for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(prm.out) + obase + cb);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint32_t w[4];
+              for (int i = 0; i < 4; ++i) {
+                uint32_t w[4];
 #pragma unroll
-              for (int k2 = 0; k2 < 4; ++k2)
-                w[k2] = float_to_bf16_bits(r[8 * i + 2 * k2]) | (float_to_bf16_bits(r[8 * i + 2 * k2 + 1]) << 16);
-              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int k2 = 0; k2 < 4; ++k2)
+                  w[k2] = float_to_bf16_bits(r[8 * i + 2 * k2]) | (float_to_bf16_bits(r[8 * i + 2 * k2 + 1]) << 16);
+                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
             }
           }
         }
+        if (prm.lse && half == 0 && qrow < prm.N)
+          prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(lt) - kLog2P8) * 0.69314718055994531f;
       }
-      if (prm.lse && qrow < prm.N)
-        prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(l) - kLog2P8) * 0.69314718055994531f;
     }
   }
 

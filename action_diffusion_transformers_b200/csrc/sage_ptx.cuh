@@ -7,6 +7,12 @@
 
 namespace sage {
 
+// Two binary32 values held in one 64-bit register (first value in the low
+// word), the operand form of the sm_100 add/mul/fma.f32x2 instructions.  The
+// pair never leaves its register between operations, so no moves are needed
+// to build operand pairs.
+typedef unsigned long long f32x2_t;
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -215,6 +221,105 @@ __device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t v) {
       "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
       : "memory");
 }
+// 32 consecutive 32-bit columns, waited for and returned as 16 pairs.
+__device__ __forceinline__ void tmem_ld32_pairs(uint32_t taddr, f32x2_t (&r)[16]) {
+  asm volatile(
+      "{.reg .b32 t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "mov.b64 %0, {t0, t1};\n\t"
+      "mov.b64 %1, {t2, t3};\n\t"
+      "mov.b64 %2, {t4, t5};\n\t"
+      "mov.b64 %3, {t6, t7};\n\t"
+      "mov.b64 %4, {t8, t9};\n\t"
+      "mov.b64 %5, {t10, t11};\n\t"
+      "mov.b64 %6, {t12, t13};\n\t"
+      "mov.b64 %7, {t14, t15};\n\t"
+      "mov.b64 %8, {t16, t17};\n\t"
+      "mov.b64 %9, {t18, t19};\n\t"
+      "mov.b64 %10, {t20, t21};\n\t"
+      "mov.b64 %11, {t22, t23};\n\t"
+      "mov.b64 %12, {t24, t25};\n\t"
+      "mov.b64 %13, {t26, t27};\n\t"
+      "mov.b64 %14, {t28, t29};\n\t"
+      "mov.b64 %15, {t30, t31};\n\t"
+      "}"
+      : "=l"(r[0]), "=l"(r[1]), "=l"(r[2]), "=l"(r[3]), "=l"(r[4]), "=l"(r[5]), "=l"(r[6]), "=l"(r[7]), "=l"(r[8]), "=l"(r[9]), "=l"(r[10]), "=l"(r[11]), "=l"(r[12]), "=l"(r[13]), "=l"(r[14]), "=l"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// Store 16 pairs into 32 consecutive 32-bit TMEM columns (low word first);
+// completion is awaited with tmem_wait_st().
+__device__ __forceinline__ void tmem_st32_pairs(uint32_t taddr, const f32x2_t (&r)[16]) {
+  asm volatile(
+      "{.reg .b32 t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31;\n\t"
+      "mov.b64 {t0, t1}, %1;\n\t"
+      "mov.b64 {t2, t3}, %2;\n\t"
+      "mov.b64 {t4, t5}, %3;\n\t"
+      "mov.b64 {t6, t7}, %4;\n\t"
+      "mov.b64 {t8, t9}, %5;\n\t"
+      "mov.b64 {t10, t11}, %6;\n\t"
+      "mov.b64 {t12, t13}, %7;\n\t"
+      "mov.b64 {t14, t15}, %8;\n\t"
+      "mov.b64 {t16, t17}, %9;\n\t"
+      "mov.b64 {t18, t19}, %10;\n\t"
+      "mov.b64 {t20, t21}, %11;\n\t"
+      "mov.b64 {t22, t23}, %12;\n\t"
+      "mov.b64 {t24, t25}, %13;\n\t"
+      "mov.b64 {t26, t27}, %14;\n\t"
+      "mov.b64 {t28, t29}, %15;\n\t"
+      "mov.b64 {t30, t31}, %16;\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31};\n\t"
+      "}"
+      :
+      : "r"(taddr), "l"(r[0]), "l"(r[1]), "l"(r[2]), "l"(r[3]), "l"(r[4]), "l"(r[5]), "l"(r[6]), "l"(r[7]), "l"(r[8]), "l"(r[9]), "l"(r[10]), "l"(r[11]), "l"(r[12]), "l"(r[13]), "l"(r[14]), "l"(r[15])
+      : "memory");
+}
+// 64 consecutive 32-bit columns of this warp's 32 TMEM lanes, waited for and
+// returned as 32 pairs (column 2i in the low word of r[i]).  The wait is inside
+// the same asm statement, so the pairs are never read before the load lands.
+__device__ __forceinline__ void tmem_ld64_pairs(uint32_t taddr, f32x2_t (&r)[32]) {
+  asm volatile(
+      "{.reg .b32 t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31, t32, t33, t34, t35, t36, t37, t38, t39, t40, t41, t42, t43, t44, t45, t46, t47, t48, t49, t50, t51, t52, t53, t54, t55, t56, t57, t58, t59, t60, t61, t62, t63;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31, t32, t33, t34, t35, t36, t37, t38, t39, t40, t41, t42, t43, t44, t45, t46, t47, t48, t49, t50, t51, t52, t53, t54, t55, t56, t57, t58, t59, t60, t61, t62, t63}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "mov.b64 %0, {t0, t1};\n\t"
+      "mov.b64 %1, {t2, t3};\n\t"
+      "mov.b64 %2, {t4, t5};\n\t"
+      "mov.b64 %3, {t6, t7};\n\t"
+      "mov.b64 %4, {t8, t9};\n\t"
+      "mov.b64 %5, {t10, t11};\n\t"
+      "mov.b64 %6, {t12, t13};\n\t"
+      "mov.b64 %7, {t14, t15};\n\t"
+      "mov.b64 %8, {t16, t17};\n\t"
+      "mov.b64 %9, {t18, t19};\n\t"
+      "mov.b64 %10, {t20, t21};\n\t"
+      "mov.b64 %11, {t22, t23};\n\t"
+      "mov.b64 %12, {t24, t25};\n\t"
+      "mov.b64 %13, {t26, t27};\n\t"
+      "mov.b64 %14, {t28, t29};\n\t"
+      "mov.b64 %15, {t30, t31};\n\t"
+      "mov.b64 %16, {t32, t33};\n\t"
+      "mov.b64 %17, {t34, t35};\n\t"
+      "mov.b64 %18, {t36, t37};\n\t"
+      "mov.b64 %19, {t38, t39};\n\t"
+      "mov.b64 %20, {t40, t41};\n\t"
+      "mov.b64 %21, {t42, t43};\n\t"
+      "mov.b64 %22, {t44, t45};\n\t"
+      "mov.b64 %23, {t46, t47};\n\t"
+      "mov.b64 %24, {t48, t49};\n\t"
+      "mov.b64 %25, {t50, t51};\n\t"
+      "mov.b64 %26, {t52, t53};\n\t"
+      "mov.b64 %27, {t54, t55};\n\t"
+      "mov.b64 %28, {t56, t57};\n\t"
+      "mov.b64 %29, {t58, t59};\n\t"
+      "mov.b64 %30, {t60, t61};\n\t"
+      "mov.b64 %31, {t62, t63};\n\t"
+      "}"
+      : "=l"(r[0]), "=l"(r[1]), "=l"(r[2]), "=l"(r[3]), "=l"(r[4]), "=l"(r[5]), "=l"(r[6]), "=l"(r[7]), "=l"(r[8]), "=l"(r[9]), "=l"(r[10]), "=l"(r[11]), "=l"(r[12]), "=l"(r[13]), "=l"(r[14]), "=l"(r[15]), "=l"(r[16]), "=l"(r[17]), "=l"(r[18]), "=l"(r[19]), "=l"(r[20]), "=l"(r[21]), "=l"(r[22]), "=l"(r[23]), "=l"(r[24]), "=l"(r[25]), "=l"(r[26]), "=l"(r[27]), "=l"(r[28]), "=l"(r[29]), "=l"(r[30]), "=l"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // After tmem_wait_ld(): ties the loaded registers to this point, so that no use
 // of them is scheduled between the asynchronous tcgen05.ld and its wait.
@@ -225,11 +330,6 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- numerics
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 // Two floats -> two E4M3 bytes (round to nearest even, saturate to +-448);
 // `lo` lands in bits 0..7, `hi` in bits 8..15.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
@@ -315,30 +415,116 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
-// 2^x for a pair, on the FMA pipe instead of the MUFU unit.  Cody-Waite style
-// split x = n + f with n = round(x) (the 1.5*2^23 addition leaves n in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f from a quintic fitted for minimax
-// relative error on [-1/2, 1/2] (coefficients from a linear-programming fit;
-// 2.2e-7 relative error after FP32 Horner evaluation, about the accuracy of the
-// hardware ex2.approx); n is added to the exponent field.  x is clamped to
-// >= -125 so the exponent stays normal (2^-125 is far below what an E4M3 code
-// or the row sum can resolve).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 xr = fadd2(x, make_float2(kRound, kRound));
-  const float2 nf = fadd2(xr, make_float2(-kRound, -kRound));
-  const float2 f = ffma2(nf, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(0.0013185542775318027f, 0.0013185542775318027f), f,
-                   make_float2(0.009675252251327038f, 0.009675252251327038f));
-  p = ffma2(p, f, make_float2(0.055510472506284714f, 0.055510472506284714f));
-  p = ffma2(p, f, make_float2(0.24022142589092255f, 0.24022142589092255f));
-  p = ffma2(p, f, make_float2(0.6931467056274414f, 0.6931467056274414f));
-  p = ffma2(p, f, make_float2(1.0f, 1.0f));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(xr.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(xr.y) << 23)));
+// ---------------------------------------------------------------- FP32 pairs
+// (f32x2_t, declared at the top of this file.)
+
+__device__ __forceinline__ f32x2_t x2_splat(float v) {
+  f32x2_t d;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(d) : "f"(v));
+  return d;
+}
+__device__ __forceinline__ f32x2_t x2_add(f32x2_t a, f32x2_t b) {
+  f32x2_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2_t x2_sub(f32x2_t a, f32x2_t b) {
+  f32x2_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2_t x2_mul(f32x2_t a, f32x2_t b) {
+  f32x2_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2_t x2_fma(f32x2_t a, f32x2_t b, f32x2_t c) {
+  f32x2_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float x2_lo(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float x2_hi(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+// Per 32-bit word: bits(p) + (bits(xr) << 23), i.e. the integer in the low bits
+// of xr added to the exponent field of p.
+__device__ __forceinline__ f32x2_t x2_add_exponent(f32x2_t p, f32x2_t xr) {
+  f32x2_t d;
+  asm("{.reg .b32 pl, ph, xl, xh;\n\t"
+      "mov.b64 {pl, ph}, %1;\n\tmov.b64 {xl, xh}, %2;\n\t"
+      "shl.b32 xl, xl, 23;\n\tshl.b32 xh, xh, 23;\n\t"
+      "add.u32 pl, pl, xl;\n\tadd.u32 ph, ph, xh;\n\t"
+      "mov.b64 %0, {pl, ph};}"
+      : "=l"(d) : "l"(p), "l"(xr));
+  return d;
+}
+// Four binary32 values (two pairs) -> four E4M3 bytes, round to nearest even,
+// saturating to +-448; a.lo lands in bits 0..7, a.hi 8..15, b.lo 16..23, b.hi 24..31.
+__device__ __forceinline__ uint32_t x2_e4m3x4(f32x2_t a, f32x2_t b) {
+  uint32_t d;
+  asm("{.reg .f32 al, ah, bl, bh;\n\t.reg .b16 ca, cb;\n\t"
+      "mov.b64 {al, ah}, %1;\n\tmov.b64 {bl, bh}, %2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 ca, ah, al;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 cb, bh, bl;\n\t"
+      "mov.b32 %0, {ca, cb};}"
+      : "=r"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x with every step a binary32 operation whose rounding is fixed, so that the
+// result is reproducible bit for bit on any IEEE machine (the CPU oracle runs
+// the same steps): Cody-Waite split x = n + f with n = round(x) by the
+// 1.5 * 2^23 addition (which leaves n, two's complement, in the low bits of
+// xr), f = x - n exactly, 2^f from a degree-5 polynomial with c0 = 1 fitted
+// for minimax relative error on [-1/2, 1/2] (linear programming; 2.2e-7 after
+// binary32 Horner evaluation with fused multiply-adds), and n added to the
+// exponent field of the polynomial's value: exactly p * 2^n for n >= -125.
+// Requires x >= -126 (callers clamp).
+constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
+constexpr float kExp2C0 = 1.0f;
+constexpr float kExp2C1 = 0.6931465864181519f;
+constexpr float kExp2C2 = 0.24022166430950165f;
+constexpr float kExp2C3 = 0.055510472506284714f;
+constexpr float kExp2C4 = 0.009674952365458012f;
+constexpr float kExp2C5 = 0.0013202981790527701f;
+constexpr float kExp2Min = -126.0f;
+
+// The constant pairs of exp2_fixed_x2, built once per thread.
+struct Exp2Consts {
+  f32x2_t round, c0, c1, c2, c3, c4, c5;
+  __device__ __forceinline__ Exp2Consts()
+      : round(x2_splat(kExp2Round)), c0(x2_splat(kExp2C0)), c1(x2_splat(kExp2C1)), c2(x2_splat(kExp2C2)),
+        c3(x2_splat(kExp2C3)), c4(x2_splat(kExp2C4)), c5(x2_splat(kExp2C5)) {}
+};
+
+__device__ __forceinline__ f32x2_t exp2_fixed_x2(f32x2_t x, const Exp2Consts& k) {
+  const f32x2_t xr = x2_add(x, k.round);
+  const f32x2_t nf = x2_sub(xr, k.round);
+  const f32x2_t f = x2_sub(x, nf);
+  f32x2_t p = x2_fma(k.c5, f, k.c4);
+  p = x2_fma(p, f, k.c3);
+  p = x2_fma(p, f, k.c2);
+  p = x2_fma(p, f, k.c1);
+  p = x2_fma(p, f, k.c0);
+  return x2_add_exponent(p, xr);
+}
+// Scalar form, clamping x at -126 itself.
+__device__ __forceinline__ float exp2_fixed(float x) {
+  x = fmaxf(x, kExp2Min);
+  const float xr = __fadd_rn(x, kExp2Round);
+  const float nf = __fadd_rn(xr, -kExp2Round);
+  const float f = __fsub_rn(x, nf);
+  float p = __fmaf_rn(kExp2C5, f, kExp2C4);
+  p = __fmaf_rn(p, f, kExp2C3);
+  p = __fmaf_rn(p, f, kExp2C2);
+  p = __fmaf_rn(p, f, kExp2C1);
+  p = __fmaf_rn(p, f, kExp2C0);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(xr) << 23));
 }
 
 }  // namespace sage

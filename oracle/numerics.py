@@ -88,6 +88,35 @@ def f64_to_f32(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float32)
 
 
+def fma32(a, b, c) -> np.ndarray:
+    """IEEE binary32 fused multiply-add: RNE of the exact a*b + c, one rounding.
+
+    a, b, c are float32 values (any array-like; broadcast).  The product of two
+    binary32 numbers has at most 48 significant bits, so it is exact in
+    float64.  The sum is taken in float64 together with its exact error
+    (Knuth's TwoSum), and the float64 sum is rounded to binary32.  That double
+    rounding can only go wrong when the float64 sum lies exactly on a binary32
+    midpoint while the exact sum does not; then the error term's sign picks
+    the neighbour the exact sum is closer to.
+    """
+    a64 = np.asarray(a, dtype=np.float32).astype(np.float64)
+    b64 = np.asarray(b, dtype=np.float32).astype(np.float64)
+    c64 = np.asarray(c, dtype=np.float32).astype(np.float64)
+    p = a64 * b64                                   # exact
+    s = p + c64
+    bv = s - p
+    err = (p - (s - bv)) + (c64 - bv)               # exact: p + c == s + err
+    r = s.astype(np.float32)
+    with np.errstate(invalid="ignore", over="ignore"):
+        r64 = r.astype(np.float64)
+        d = s - r64                                 # exact: r is a binary32 neighbour of s
+        toward = np.where(d > 0, np.float32(np.inf), np.float32(-np.inf))
+        nxt = np.nextafter(r, toward)
+        mid = np.isfinite(r64) & (d != 0) & (2.0 * d == nxt.astype(np.float64) - r64)
+        fix = mid & (np.sign(err) == np.sign(d)) & (err != 0)
+    return np.where(fix, nxt, r).astype(np.float32)
+
+
 # ----------------------------------------------------------------------------
 # E4M3 (FP8)
 # ----------------------------------------------------------------------------

@@ -27,9 +27,12 @@ for |sum| < 2**53.
 Parity status: pinned by tests/test_oracle_sage.py (quantizers by brute force
 and invariants; the attention tile loop by running it with quantization off
 against brute-force FP64 softmax attention; smoothing by the softmax shift
-invariance; closed forms for degenerate inputs).  The exp2 of the FP32 softmax
-is evaluated in FP64 and rounded once; the GPU's hardware exp2 is not
-bit-matched by design, which is why attention parity has a tolerance.
+invariance; closed forms for degenerate inputs; the softmax exp2 against
+numpy's exp2 within its stated error bound and exactly at integers; the fused
+multiply-add against exact rational rounding).  With the exp2 and the FMA
+fixed by the contract, the E4M3 codes of P are reproducible; attention parity
+keeps a tolerance for the tensor core's FP32 summation order and the order of
+the row-sum additions.
 """
 from __future__ import annotations
 
@@ -38,7 +41,7 @@ import math
 import numpy as np
 
 from .numerics import (bf16_bits_to_f32, e4m3_decode, e4m3_encode,
-                       f32_to_bf16_bits, f64_to_bf16_bits, rn32,
+                       f32_to_bf16_bits, f64_to_bf16_bits, fma32, rn32,
                        round_f32_to_bf16)
 
 QK_BLOCK = 64        # tokens per INT8 scale block of Q and K
@@ -48,6 +51,7 @@ SUM_LANES = 32       # interleaved second-level partial sums
 INT8_MAX = 127.0
 E4M3_MAX = 448.0
 LOG2E = 1.4426950408889634
+LOG2_P_UNIT = np.float32(math.log2(E4M3_MAX))   # RN32(log2 448), the P scale in the exponent
 
 
 def npad(n: int) -> int:
@@ -206,33 +210,76 @@ def quant_v(v_bits: np.ndarray):
 # ----------------------------------------------------------------------------
 # A6-A10: tiled attention with FP32 online softmax
 # ----------------------------------------------------------------------------
+# exp2 of the FP32 softmax (reading: the pages fix FP32 for the softmax but not
+# how exp2 is evaluated; this contract fixes it so that every P8 code is
+# reproducible).  Cody-Waite split with round-to-nearest, then a degree-5
+# polynomial with c0 = 1 fitted for minimax relative error on [-1/2, 1/2]
+# (oracle/fit_exp2.py; 2.2e-7 after binary32 evaluation), then n added to the
+# exponent field.
+EXP2_C = tuple(np.float32(v) for v in (1.0, 0.6931465864181519, 0.24022166430950165,
+                                       0.055510472506284714, 0.009674952365458012,
+                                       0.0013202981790527701))
+EXP2_MIN = np.float32(-126.0)
+EXP2_ROUND = np.float32(12582912.0)   # 1.5 * 2^23
+
+
+def exp2_contract(u) -> np.ndarray:
+    """2^u as the contract evaluates it, every step a binary32 operation.
+
+      x  = max(u, -126)
+      xr = RN(x + 1.5 * 2^23)           the integer n = round(x) in the low bits (two's complement)
+      nf = RN(xr - 1.5 * 2^23)          = n, exactly
+      f  = RN(x - nf)                   exact, |f| <= 1/2
+      p  = c5; p = fma(p, f, c_k) for k = 4 .. 0
+      y  = the binary32 whose bits are bits(p) + (bits(xr) << 23) mod 2^32,
+           i.e. n added to the exponent field of p: exactly p * 2^n for
+           n >= -125 (p lies in [2^-1/2, 2^1/2]); at n = -126 a value below
+           2^-125 that no E4M3 code or row sum can tell from 0.
+    """
+    x = np.maximum(np.asarray(u, dtype=np.float32), EXP2_MIN)
+    xr = rn32(x.astype(np.float64) + np.float64(EXP2_ROUND))
+    nf = rn32(xr.astype(np.float64) - np.float64(EXP2_ROUND))
+    f = rn32(x.astype(np.float64) - nf.astype(np.float64))
+    p = np.full(f.shape, EXP2_C[5], dtype=np.float32)
+    for k in (4, 3, 2, 1, 0):
+        p = fma32(p, f, EXP2_C[k])
+    bits = p.view(np.uint32) + (xr.view(np.uint32) << np.uint32(23))   # uint32 arithmetic wraps
+    return bits.astype(np.uint32).view(np.float32)
+
+
 def _identity(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, quant_p,
-                 p_unit, two_pass=False):
+def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, quant_p,
+                 log2_p_unit, two_pass=False):
     """Online-softmax attention over 128-key tiles for one (b, h).
 
     S         [R, >= n_keys] float64: exact score numerators (INT32 dot
               products, or FP64 dot products with quantization off).
-    col_mult  f(j0, j1) -> [R, j1 - j0] multipliers taking S into the exp2
+    col_mult  f(j0, j1) -> [R, j1 - j0] multipliers c taking S into the exp2
               domain (dequant scales x sm_scale x log2 e).
     Vt        [D, >= n_keys] float64: the (centred, dequantized-code) values.
-    out_mult  [D] per-channel output factor (V scale / p_unit); out_add [D]
-              the V mean added back.
+    out_mult  [D] per-channel output factor (the V scale); out_add [D] the V
+              mean added back.
     rn        rounding applied after every step (rn32, or identity in FP64).
-    quant_p   P quantizer applied to p * p_unit (E4M3 round trip, or identity).
+    fma       fused multiply-add with one rounding (fma32, or exact in FP64).
+    exp2      the exp2 of the softmax (exp2_contract, or np.exp2 in FP64).
+    quant_p   P quantizer (E4M3 round trip, or identity).
+    log2_p_unit  log2 of the P scale folded into the exponent: RN32(log2 448)
+              with quantization on, 0 with it off.
 
     Per tile j (keys j0..j1-1, those >= n_keys excluded):
-      t     = rn(S * c)                          A7 dequant
-      m_new = max(m, max_k t)
-      alpha = rn(exp2(rn(m - m_new)))            (0 on the first tile)
-      p     = rn(exp2(rn(t - m_new)))            P~ in [0, 1]
-      l     = rn(rn(l * alpha) + rn(sum_k p))    row sum of UNquantized P~
-      P8    = quant_p(rn(p * p_unit))            A8
-      acc   = rn(rn(acc * alpha) + rn(P8 @ V))   A9, product sum exact then rounded
-    Epilogue (A10): o = rn(rn(rn(acc * out_mult) * rn(1 / l)) + out_add).
+      t     = rn(S * c)                          scores in the exp2 domain
+      m_new = max(m, max_k t)                    running row max
+      alpha = exp2(rn(m - m_new))                (~0 on the first tile, m = -inf)
+      e     = rn(log2_p_unit - m_new)
+      y     = exp2(fma(S, c, e))                 = P~ * 448, P~ = exp2(t - m_new)
+      l     = rn(rn(l * alpha) + rn(sum_k y))    row sum of the unquantized y
+      P8    = quant_p(y)                         E4M3 code of P~ * 448
+      acc   = rn(rn(acc * alpha) + rn(P8 @ V))   product sum exact, then rounded
+    Epilogue: o = fma(rn(acc * out_mult), rn(1 / l), out_add); the P scale
+    cancels between acc and l.
     two_pass: m is the final row max from the start (alpha = 1 throughout).
     Returns (o [R, D], m [R], l [R]).
     """
@@ -249,19 +296,26 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, quant_p,
     acc = np.zeros((R, D))
     for j in range(nkv):
         j0, j1 = j * TILE, min(n_keys, (j + 1) * TILE)
-        t = rn(S[:, j0:j1] * col_mult(j0, j1))
+        c = col_mult(j0, j1)
+        t = rn(S[:, j0:j1] * c)
         m_new = m if two_pass else np.maximum(m, t.max(axis=1))
         with np.errstate(invalid="ignore"):
-            alpha = np.where(np.isneginf(m), 0.0, rn(np.exp2(rn(m - m_new))))
+            alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2(rn(m - m_new)), dtype=np.float64))
         if two_pass:
             alpha = np.ones(R)
-        p = rn(np.exp2(rn(t - m_new[:, None])))
-        l = rn(rn(l * alpha) + rn(p.sum(axis=1)))
-        p8 = quant_p(rn(p * p_unit))
+        e = rn(log2_p_unit - m_new)
+        y = np.asarray(exp2(fma(S[:, j0:j1], c, e[:, None])), dtype=np.float64)
+        l = rn(rn(l * alpha) + rn(y.sum(axis=1)))
+        p8 = quant_p(y)
         acc = rn(rn(acc * alpha[:, None]) + rn(p8 @ Vt[:, j0:j1].T))
         m = m_new
-    o = rn(rn(rn(acc * out_mult[None, :]) * rn(1.0 / l)[:, None]) + out_add[None, :])
+    o = np.asarray(fma(rn(acc * out_mult[None, :]), rn(1.0 / l)[:, None], out_add[None, :]),
+                   dtype=np.float64)
     return o, m, l
+
+
+def _fma_exact(a, b, c):
+    return np.asarray(a, np.float64) * b + c
 
 
 def _e4m3_round_trip(x):
@@ -285,8 +339,10 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     v_codes_t uint8 E4M3 [B, H, D, Npad]; v_scale, v_mean f32 [B, H, D].
     Score dequant multiplier for query row i and key j:
         c = RN32(RN32(qs[i // 64] * ks[j // 64]) * RN32(sm_scale * log2 e)),
-    the P scale is 448 (P8 = E4M3(P~ * 448)) and the output factor is
-    RN32(v_scale / 448).  sm_scale None or <= 0 means 1/sqrt(D).
+    the P scale 448 enters the exponent as RN32(log2 448) (P8 = E4M3(P~ * 448),
+    with the exponent of P~ * 448 formed by one fused multiply-add), the row
+    sum holds P~ * 448 and the output factor is the V scale itself.
+    sm_scale None or <= 0 means 1/sqrt(D).
     rows: optional query-row indices (< N) to evaluate; heads: optional list of
     (b, h) pairs.  Returns float32 [B, R, H, D] (unevaluated heads stay 0),
     plus lse [B, H, R] (natural log of the softmax denominator) if asked.
@@ -300,7 +356,6 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     out = np.zeros((B, R, H, D), dtype=np.float32)
     lse = np.zeros((B, H, R), dtype=np.float32)
     heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
-    out_mult = None
     for b, h in heads:
         Qf = q_codes[b, h, rows].astype(np.float64)
         Kf = k_codes[b, h, :N].astype(np.float64)
@@ -313,12 +368,11 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
             return rn32(rn32(qs[:, None].astype(np.float64) * kk[None, :]) * np.float64(sl2e))
 
         Vt = e4m3_decode(v_codes_t[b, h, :, :N])
-        out_mult = rn32(np.float64(v_scale[b, h]) / E4M3_MAX)
-        o, m, l = _attend_rows(S, col_mult, Vt, out_mult.astype(np.float64),
-                               v_mean[b, h].astype(np.float64), N, rn32,
-                               _e4m3_round_trip, E4M3_MAX, two_pass=two_pass)
+        o, m, l = _attend_rows(S, col_mult, Vt, v_scale[b, h].astype(np.float64),
+                               v_mean[b, h].astype(np.float64), N, rn32, fma32, exp2_contract,
+                               _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass)
         out[b, :, h, :] = o
-        lse[b, h] = rn32((m + np.log2(l)) * math.log(2.0))
+        lse[b, h] = rn32((m + np.log2(l) - math.log2(E4M3_MAX)) * math.log(2.0))
     return (out, lse) if want_lse else out
 
 
@@ -348,7 +402,7 @@ def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
         mean = V.mean(axis=0) if smooth_v else np.zeros(D)
         S = Q @ K.T
         o, _, _ = _attend_rows(S, lambda j0, j1: c, (V - mean).T, np.ones(D), mean,
-                               N, _identity, _identity, 1.0)
+                               N, _identity, _fma_exact, np.exp2, _identity, 0.0)
         out[b, :, h, :] = o
     return out
 

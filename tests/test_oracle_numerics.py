@@ -140,3 +140,67 @@ def test_e4m3_saturates_and_roundtrips():
     assert np.all(nm.e4m3_encode(-big) == 0xFE)
     codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
     assert np.array_equal(nm.e4m3_encode(nm.e4m3_decode(codes).astype(np.float32)), codes)
+
+
+def _exact_f32(x: Fraction) -> float:
+    """Reference: RNE of an exact rational onto the binary32 grid."""
+    if x == 0:
+        return 0.0
+    ax = abs(x)
+    E = math.floor(math.log2(float(ax))) if float(ax) > 0 else -200
+    while Fraction(2) ** E > ax:
+        E -= 1
+    while Fraction(2) ** (E + 1) <= ax:
+        E += 1
+    E = max(E, -126)
+    q = _exact_rne(ax, Fraction(2) ** (E - 23))
+    if q >= Fraction(2) ** 128:
+        return math.copysign(math.inf, x)
+    return float(q) if x > 0 else -float(q)
+
+
+def _fma_cases():
+    rng = np.random.default_rng(31)
+    n = 4000
+    a = (rng.standard_normal(n) * np.exp2(rng.integers(-30, 30, n))).astype(np.float32)
+    b = (rng.standard_normal(n) * np.exp2(rng.integers(-30, 30, n))).astype(np.float32)
+    # c near -a*b (cancellation) for a third, far smaller / larger for the rest
+    c = (rng.standard_normal(n) * np.exp2(rng.integers(-60, 30, n))).astype(np.float32)
+    third = n // 3
+    c[:third] = (-(a[:third].astype(np.float64) * b[:third]) * (1 + rng.standard_normal(third) * 1e-6)
+                 ).astype(np.float32)
+    # the attention exponent: integer score * FP32 multiplier + FP32 offset
+    S = rng.integers(-2_000_000, 2_000_000, 2000).astype(np.float32)
+    cm = (rng.uniform(1e-5, 1e-3, 2000)).astype(np.float32)
+    e = (-(S.astype(np.float64) * cm) + rng.uniform(-30, 9, 2000)).astype(np.float32)
+    # constructed: a*b exactly on a binary32 midpoint, c a tiny nudge either way
+    mid_a = np.float32(3.0)
+    mid_b = np.float32(1 + 2.0 ** -23)               # 3 * (1 + 2^-23): a binary32 midpoint
+    tiny = [2.0 ** -80, -(2.0 ** -80), 2.0 ** -60, -(2.0 ** -60), 0.0]
+    ca = np.full(len(tiny), mid_a, np.float32)
+    cb = np.full(len(tiny), mid_b, np.float32)
+    cc = np.asarray(tiny, np.float32)
+    A = np.concatenate([a, S, ca, -ca])
+    Bv = np.concatenate([b, cm, cb, cb])
+    C = np.concatenate([c, e, cc, cc])
+    return A, Bv, C
+
+
+def test_fma32_matches_exact_rational_rounding():
+    A, Bv, C = _fma_cases()
+    got = nm.fma32(A, Bv, C)
+    ref = np.asarray([_exact_f32(Fraction(float(x)) * Fraction(float(y)) + Fraction(float(z)))
+                      for x, y, z in zip(A, Bv, C)], dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_fma32_single_rounding_differs_from_separate_steps():
+    # 3 * (1 + 2^-23) = 3 + 2^-22 + 2^-23 is a binary32 midpoint; a nudge of
+    # -2^-80 makes the exact sum round down, which a product rounded first
+    # (ties to even: up) and a float64 sum rounded later (also on the midpoint)
+    # both get wrong.
+    a, b, c = np.float32(3.0), np.float32(1 + 2.0 ** -23), np.float32(-(2.0 ** -80))
+    fused = nm.fma32(a, b, c)
+    assert float(fused) == 3.0 + 2.0 ** -22
+    assert float(nm.rn32(nm.rn32(np.float64(a) * np.float64(b)) + np.float64(c))) == 3.0 + 2.0 ** -21
+    assert float(nm.rn32(np.float64(a) * np.float64(b) + np.float64(c))) == 3.0 + 2.0 ** -21

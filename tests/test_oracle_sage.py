@@ -285,4 +285,35 @@ def test_running_max_with_large_logit_gap():
     o, it = _pipeline(q, k, v)
     assert np.all(np.isfinite(o))
     dec = nm.e4m3_decode(it["v_codes_t"][0, 0, :, 10]) * it["v_scale"][0, 0] + it["v_mean"][0, 0]
-    assert np.abs(o[0, 5, 0] - dec).max() <= 1e-5
+    # The dominant key's exponent is S*c - RN(S*c) + (RN(log2 448 - m) - (log2 448 - m)):
+    # off by at most one FP32 ulp of the row max m (here ~1150), so its weight
+    # relative to the row sum moves by up to ln2 * ulp(m).
+    S = it["q_codes"][0, 0, 5].astype(np.float64) @ it["k_codes"][0, 0, 10].astype(np.float64)
+    c = nm.rn32(nm.rn32(np.float64(it["q_scale"][0, 0, 0]) * it["k_scale"][0, 0, 0])
+                * np.float64(so.exp2_scale(so.default_sm_scale(D))))
+    m = nm.rn32(S * np.float64(c))
+    assert m > 512
+    centred = np.abs(dec - it["v_mean"][0, 0])                  # the part scaled by P8 / l
+    tol = 2 * np.spacing(np.float32(m)) * centred + 1e-6
+    assert np.all(np.abs(o[0, 5, 0] - dec) <= tol)
+
+
+def test_exp2_contract_error_bound_and_exact_points():
+    rng = np.random.default_rng(21)
+    u = np.concatenate([rng.uniform(-125, 9.5, 200000), np.arange(-125, 10) + 0.5,
+                        np.arange(-125, 10) + 0.4999999, np.linspace(-1, 1, 20001)]).astype(np.float32)
+    y = so.exp2_contract(u).astype(np.float64)
+    rel = np.abs(y / np.exp2(u.astype(np.float64)) - 1)
+    assert rel.max() <= 2.3e-7                                    # the fit's binary32 bound
+    n = np.arange(-126, 10).astype(np.float32)
+    assert np.array_equal(so.exp2_contract(n), np.exp2(n.astype(np.float64)).astype(np.float32))
+    lo = so.exp2_contract(np.array([-126.0, -300.0, -np.inf], np.float32))
+    assert np.all(lo == np.float32(2.0 ** -126))                 # clamped below at 2^-126
+    tail = so.exp2_contract(np.linspace(-126, -125, 1001).astype(np.float32)).astype(np.float64)
+    assert np.all((tail >= 0) & (tail < 2.0 ** -124))            # the n = -126 end stays tiny
+
+
+def test_exp2_contract_coefficients_come_from_the_fit():
+    fit_exp2 = pytest.importorskip("oracle.fit_exp2")
+    c = fit_exp2.fit()
+    assert np.allclose(c, np.asarray(so.EXP2_C, np.float32), rtol=2e-6, atol=0)
