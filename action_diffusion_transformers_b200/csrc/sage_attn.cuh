@@ -1,24 +1,20 @@
 // sage_attn.cuh - quantized attention forward on sm_100a tensor cores.
 //
 // One CTA computes one 128-row query tile of one (b, h).  Warp roles:
-//   warps 0-7  softmax: two threads per query row.  Warp w reads TMEM lane
-//              quadrant w % 4 (query rows 32 (w % 4) ..) and score columns
-//              64 (w / 4) .. + 63, i.e. one 64-key scale block.  Per tile a
-//              thread loads its 64 scores once, reduces their max, swaps it
-//              with its partner thread through shared memory (an mbarrier per
-//              warp pair, so the wait is bounded), then forms E4M3 codes of
-//              P~ * 448 for its 64 keys, writes them into a 128B-swizzled
-//              shared P tile, rescales its half of the O accumulator in TMEM
-//              when the row max moves, and runs its half of the epilogue.
-//              Two CTAs share an SM, so 16 softmax warps hide each other's
-//              latencies.
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Per tile it
+//              reads its 128 scores from TMEM, reduces their max and min, forms
+//              the E4M3 codes of P~ * 448 32 keys at a time (scores re-read from
+//              TMEM, so only 32 are live next to the exp2 state), writes them
+//              into a 128B-swizzled shared P tile, rescales its row of the O
+//              accumulator in TMEM when its row max moves, and runs the
+//              epilogue.  Two CTAs share an SM.
 // S is accumulated onto the integer 0x4B400000 (the bits of 1.5 * 2^23) that
 // the softmax warps write into the S columns before each QK^T MMA: read as a
 // float, a loaded S word is then exactly 1.5 * 2^23 + S (|S| <= 127^2 * D <
 // 2^22), so one exact subtraction converts it, two at a time with f32x2.
-//   warp 8     producer: one thread issues TMA tile loads (Q once; K and V
+//   warp 4     producer: one thread issues TMA tile loads (Q once; K and V
 //              tiles into 2-stage rings).
-//   warp 9     MMA: allocates TMEM; one thread issues
+//   warp 5     MMA: allocates TMEM; one thread issues
 //              S  = Qc Kc^T  tcgen05.mma kind::i8      (INT32 accumulate)
 //              O += P8 V8    tcgen05.mma kind::f8f6f4  (FP32 accumulate).
 // TMEM (256 columns): S at columns [0, 128), O at [128, 128 + D).
@@ -42,11 +38,11 @@ namespace sage {
 
 constexpr int kBM = 128;   // query rows per tile
 constexpr int kBN = 128;   // keys per tile
-constexpr int kAttnThreads = 320;      // 8 softmax warps + producer + MMA
-constexpr int kSoftmaxThreads = 256;   // two threads per query row
-constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
-constexpr int kNumBars = 18;
+constexpr int kAttnThreads = 192;      // 4 softmax warps + producer + MMA
+constexpr int kSoftmaxThreads = 128;   // one thread per query row
+constexpr int kWarpProducer = 4;
+constexpr int kWarpMma = 5;
+constexpr int kNumBars = 14;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSBiasBits = 0x4B400000u;   // S accumulates onto these bits
 constexpr float kSBias = 12582912.0f;          // their float value, 1.5 * 2^23
@@ -66,8 +62,7 @@ struct AttnSmem {
   static constexpr int kP = kV1 + kVBytes;
   static constexpr int kVf = kP + kPBytes;     // D floats: v_scale
   static constexpr int kVm = kVf + 4 * D;      // D floats: v_mean
-  static constexpr int kX = kVm + 4 * D;       // [2 phases][2 halves][128 rows] floats: row max / sum swap
-  static constexpr int kBar = kX + 2 * 2 * kBM * 4;
+  static constexpr int kBar = kVm + 4 * D;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024; // slack for 1024-byte alignment
@@ -88,8 +83,7 @@ struct AttnParams {
 };
 
 enum : int { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
-             kBarSEmpty = 10, kBarPFull = 11, kBarPVDone = 12, kBarDrain = 13,
-             kBarPair = 14 /* 4: one per warp pair sharing a lane quadrant */ };
+             kBarSEmpty = 10, kBarPFull = 11, kBarPVDone = 12, kBarDrain = 13 };
 
 // Bounded wait whose outcome is the same in every lane of the warp, so that a
 // warp never splits in front of a warp-collective tcgen05 instruction.
@@ -103,19 +97,19 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
   return __int2float_rn(static_cast<int>(s));
 }
 
-// The contract's exponentials for 32 of this thread's keys (16 pairs of biased
-// scores s; valid counts from the first of them): u = RN(S * c + e) with e = RN(log2 448 - m_new) (one fused
-// multiply-add), y = exp2_fixed(u) = P~ * 448 -> E4M3 code; the row sum
+// The contract's exponentials for 32 of this thread's keys (biased scores s as
+// loaded from TMEM; valid counts from the first of them): u = RN(S * c + e) with e = RN(log2 448 - m_new) (one fused
+// multiply-add), y = exp2_fixed_x2(u) = P~ * 448 -> E4M3 code; the row sum
 // accumulates y.  Every step is a binary32 operation with fixed rounding, so y
 // and its code equal the oracle's bit for bit.  kClamp: some u of this warp's
 // tile may be below -126.  pk[w] holds the codes of keys 4w .. 4w+3.
 template <bool kMasked, bool kClamp>
-__device__ __forceinline__ void softmax_quarter(const f32x2_t (&s)[16], f32x2_t c2, f32x2_t e2, int valid,
+__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], f32x2_t c2, f32x2_t e2, int valid,
                                                 const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
   f32x2_t prev = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const f32x2_t sv = x2_sub(s[i], k.round);            // exact integer S (the S bias is 1.5 * 2^23 too)
+    const f32x2_t sv = x2_sub(x2_pack(s[2 * i], s[2 * i + 1]), k.round);  // exact integer S (the S bias is 1.5 * 2^23 too)
     f32x2_t u = x2_fma(sv, c2, e2);
     if (kClamp) {
       const float lo = fmaxf(x2_lo(u), kExp2Min);
@@ -136,36 +130,50 @@ __device__ __forceinline__ void softmax_quarter(const f32x2_t (&s)[16], f32x2_t 
   }
 }
 
-// Max over the valid keys and min over all keys of this thread's 64 biased scores.
+// Max over the valid keys and min over all keys of 32 biased scores.
 template <bool kMasked>
-__device__ __forceinline__ void half_minmax(const f32x2_t (&s)[32], int valid, float& mx, float& mn) {
-  float v[64];
+__device__ __forceinline__ void chunk_minmax(const uint32_t (&a)[32], int valid, float& mx, float& mn) {
+  float v[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    v[2 * i] = x2_lo(s[i]);
-    v[2 * i + 1] = x2_hi(s[i]);
-  }
-  float w[22];
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+  float w[11];
 #pragma unroll
-  for (int i = 0; i < 21; ++i) w[i] = fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  w[21] = v[63];
-  float x[8];
-#pragma unroll
-  for (int i = 0; i < 7; ++i) x[i] = fmin3(w[3 * i], w[3 * i + 1], w[3 * i + 2]);
-  x[7] = w[21];
-  mn = fminf(fmin3(x[0], x[1], x[2]), fmin3(x[3], x[4], fminf(x[5], fminf(x[6], x[7]))));
+  for (int i = 0; i < 10; ++i) w[i] = fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  w[10] = fminf(v[30], v[31]);
+  mn = fminf(fmin3(fmin3(w[0], w[1], w[2]), fmin3(w[3], w[4], w[5]), fmin3(w[6], w[7], w[8])),
+             fminf(w[9], w[10]));
   if (kMasked) {
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
+    for (int i = 0; i < 32; ++i)
       if (i >= valid) v[i] = 0.f;                        // below every biased score
   }
 #pragma unroll
-  for (int i = 0; i < 21; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  w[21] = v[63];
+  for (int i = 0; i < 10; ++i) w[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  w[10] = fmaxf(v[30], v[31]);
+  mx = fmaxf(fmax3(fmax3(w[0], w[1], w[2]), fmax3(w[3], w[4], w[5]), fmax3(w[6], w[7], w[8])),
+             fmaxf(w[9], w[10]));
+}
+
+// The exponential pass over a row's 128 scores in TMEM (taddr), 32 at a time;
+// each chunk's 32 codes go straight to
+// the row's 128B-swizzled P line (16-byte chunk q of row r lives at q ^ (r & 7)).
+// kSlow: masked keys or clamped exponents.
+template <bool kSlow>
+__device__ __forceinline__ void exp_pass(uint32_t taddr, float c0, float c1, float e, int valid,
+                                         const Exp2Consts& ek, f32x2_t (&lsum)[4], uint8_t* prow, int row) {
+  const f32x2_t e2 = x2_splat(e);
 #pragma unroll
-  for (int i = 0; i < 7; ++i) x[i] = fmax3(w[3 * i], w[3 * i + 1], w[3 * i + 2]);
-  x[7] = w[21];
-  mx = fmaxf(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], fmaxf(x[5], fmaxf(x[6], x[7]))));
+  for (int qq = 0; qq < 4; ++qq) {
+    uint32_t cur[32];
+    tmem_ld32(taddr + 32 * qq, cur);
+    tmem_wait_ld();
+    reg_fence(cur);
+    const f32x2_t c2 = x2_splat(qq < 2 ? c0 : c1);
+    uint32_t pk[8];
+    softmax_quarter<kSlow, kSlow>(cur, c2, e2, valid - 32 * qq, ek, lsum, pk);
+    *reinterpret_cast<uint4*>(prow + ((2 * qq) ^ (row & 7)) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4*>(prow + ((2 * qq + 1) ^ (row & 7)) * 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  }
 }
 
 template <int D>
@@ -199,7 +207,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     for (int i = 0; i < kNumBars; ++i) {
       uint32_t count = 1u;
       if (i == kBarSEmpty || i == kBarPFull) count = kSoftmaxThreads;
-      if (i >= kBarPair) count = 64u;
       mbar_init(&bars[i], count);
     }
     *abort_flag = 0;
@@ -310,108 +317,98 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int quad = warp & 3;                    // TMEM lane quadrant
-    const int half = warp >> 2;                   // score columns 64 half .. + 63
-    const int row = quad * 32 + lane;             // TMEM lane == query row in tile
-    constexpr int kOH = D / 2;                    // O / output columns per thread
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t ts = tmem_s + lane_base + static_cast<uint32_t>(half * 64);
-    const uint32_t to = tmem_o + lane_base + static_cast<uint32_t>(half * kOH);
-    uint64_t* pair_bar = &bars[kBarPair + quad];
-    float* xch = reinterpret_cast<float*>(smem + L::kX);   // [phase & 1][half][row]
+    const int row = tid;                          // TMEM lane == query row in tile
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t ts = tmem_s + lane_base;
+    const uint32_t to = tmem_o + lane_base;
     const int nqb = prm.Npad / 64;
     const float qs = prm.q_scale[static_cast<int64_t>(bh) * nqb + qt * 2 + (row >> 6)];
-    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * nqb + half;  // this half's key block
+    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * nqb;
     const float sl2e = prm.sl2e;
     uint8_t* sP = smem + L::kP;
     const float kNegInf = -__int_as_float(0x7F800000);
     float m = kNegInf;
-    float l = 0.f;                                // this half's sum of P~ * 448
+    float l = 0.f;                                // sum of P~ * 448
     bool ok = true;
     const Exp2Consts ek;
     static_assert(kSBias == kExp2Round, "the S bias doubles as the exp2 rounding constant");
-    // Seed this thread's S columns with the bias and release them for the first QK^T MMA.
-    tmem_st32_fill(ts, kSBiasBits);
-    tmem_st32_fill(ts + 32, kSBiasBits);
+    // Seed S with the bias and release it for the first QK^T MMA.
+    tmem_fill64(ts, kSBiasBits);
+    tmem_fill64(ts + 64, kSBiasBits);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&bars[kBarSEmpty]);
     for (int j = 0; j < nkv; ++j) {
-      const float c = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
+      // Keys 0-63 and 64-127 of the tile are two scale blocks.
+      const float c0 = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
+      const float c1 = __fmul_rn(__fmul_rn(qs, ks[2 * j + 1]), sl2e);
       if (!warp_wait(&bars[kBarSFull], static_cast<uint32_t>(j) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int valid = min(kBN, prm.N - j * kBN) - half * 64;   // valid keys among this thread's 64
-      f32x2_t sp[32];                             // this thread's 64 biased scores
-      tmem_ld64_pairs(ts, sp);
-      // This half's max of t = RN(S * c) (c > 0, so it is the max S scaled), -inf if
-      // no key; and its min S, which bounds every u from below.
-      float th, smin;
+      const int valid = min(kBN, prm.N - j * kBN);   // valid keys in this tile
+      // Row max of t = RN(S * c) (c > 0, so per block it is the max S scaled) and
+      // the per-block min S, which bounds every u from below.
+      float tmax, smin0, smin1;
       {
-        float mx, mn;
-        if (valid >= 64)
-          half_minmax<false>(sp, 64, mx, mn);
-        else
-          half_minmax<true>(sp, valid, mx, mn);
-        th = __fmul_rn(__fsub_rn(mx, kSBias), c);
-        if (valid <= 0) th = kNegInf;
-        smin = __fsub_rn(mn, kSBias);
+        // Four 32-column loads, each issued while the previous chunk is reduced.
+        uint32_t ra[32], rb[32];
+        float mx[4], mn[4];
+        tmem_ld32(ts, ra);
+        tmem_wait_ld();
+        reg_fence(ra);
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          uint32_t (&cur)[32] = (qq & 1) ? rb : ra;
+          uint32_t (&nxt)[32] = (qq & 1) ? ra : rb;
+          if (qq < 3) tmem_ld32(ts + 32 * (qq + 1), nxt);
+          if (valid >= kBN)
+            chunk_minmax<false>(cur, 32, mx[qq], mn[qq]);
+          else
+            chunk_minmax<true>(cur, valid - 32 * qq, mx[qq], mn[qq]);
+          if (qq < 3) {
+            tmem_wait_ld();
+            reg_fence(nxt);
+          }
+        }
+        tmax = __fmul_rn(__fsub_rn(fmaxf(mx[0], mx[1]), kSBias), c0);
+        if (valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(fmaxf(mx[2], mx[3]), kSBias), c1));
+        smin0 = __fsub_rn(fminf(mn[0], mn[1]), kSBias);
+        smin1 = __fsub_rn(fminf(mn[2], mn[3]), kSBias);
       }
-      float* xp = xch + (j & 1) * (2 * kBM);
-      xp[half * kBM + row] = th;
-      mbar_arrive(pair_bar);
-      if (!warp_wait(pair_bar, static_cast<uint32_t>(j) & 1, abort_flag, tmo)) {
+      const float m_new = fmaxf(m, tmax);
+      const float alpha = exp2_fixed5(__fsub_rn(m, m_new));
+      const float e = __fsub_rn(kLog2P8, m_new);
+      // u is monotone in S (c > 0), so the smallest u of a block is its min S's;
+      // clamping is the identity unless that is below -126.
+      const bool clamp = __any_sync(0xFFFFFFFFu, fminf(__fmaf_rn(smin0, c0, e), __fmaf_rn(smin1, c1, e)) < kExp2Min);
+      // P is single-buffered in shared memory: PV_{j-1} (issued right after QK_j)
+      // must have read it before this tile's codes are written.
+      if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) {
         ok = false;
         break;
       }
-      const float m_new = fmaxf(m, fmaxf(th, xp[(half ^ 1) * kBM + row]));
-      const float alpha = exp2_fixed(__fsub_rn(m, m_new));
-      const float e = __fsub_rn(kLog2P8, m_new);
-      // u is monotone in S (c > 0), so the smallest u is the min S's; clamping is
-      // the identity unless it is below -126.
-      const bool clamp = __any_sync(0xFFFFFFFFu, __fmaf_rn(smin, c, e) < kExp2Min);
-      uint32_t pk[16];  // this thread's 64 E4M3 codes, 4 per word, key order
       f32x2_t lsum[4] = {0, 0, 0, 0};
-      const f32x2_t c2 = x2_splat(c);
-      const f32x2_t e2 = x2_splat(e);
-      // Scores again, 32 at a time, so that only 32 are live with the exp2 state.
-#pragma unroll
-      for (int qq = 0; qq < 2; ++qq) {
-        f32x2_t sq[16];
-        tmem_ld32_pairs(ts + 32 * qq, sq);
-        if (valid >= 64 && !clamp)
-          softmax_quarter<false, false>(sq, c2, e2, 64, ek, lsum, pk + 8 * qq);
-        else
-          softmax_quarter<true, true>(sq, c2, e2, valid - 32 * qq, ek, lsum, pk + 8 * qq);
-      }
+      uint8_t* prow = sP + row * 128;
+      if (valid >= kBN && !clamp)
+        exp_pass<false>(ts, c0, c1, e, kBN, ek, lsum, prow, row);
+      else
+        exp_pass<true>(ts, c0, c1, e, valid, ek, lsum, prow, row);
       // Re-seed S with the bias for the next tile's MMA, then release the buffer.
-      tmem_st32_fill(ts, kSBiasBits);
-      tmem_st32_fill(ts + 32, kSBiasBits);
+      tmem_fill64(ts, kSBiasBits);
+      tmem_fill64(ts + 64, kSBiasBits);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[kBarSEmpty]);
       const f32x2_t ls2 = x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
       l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(x2_lo(ls2), x2_hi(ls2)));
 
-      if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) {
-        ok = false;
-        break;
-      }
-      // P row -> shared tile, 128B swizzle: 16-byte chunk q of row r lives at q ^ (r & 7).
-      uint8_t* prow = sP + row * 128;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int pc = (half * 4 + cc) ^ (row & 7);
-        *reinterpret_cast<uint4*>(prow + pc * 16) =
-            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      }
       if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
         tc_fence_after();
         const f32x2_t a2 = x2_splat(alpha);
 #pragma unroll
-        for (int cb = 0; cb < kOH; cb += 32) {
+        for (int cb = 0; cb < D; cb += 32) {
           f32x2_t o[16];
           tmem_ld32_pairs(to + cb, o);
 #pragma unroll
@@ -426,56 +423,47 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       m = m_new;
     }
     if (ok && warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(nkv - 1) & 1, abort_flag, tmo)) {
-      // Row sum: the two halves' sums, added in a fixed order by both threads.
-      float* xp = xch + (nkv & 1) * (2 * kBM);
-      xp[half * kBM + row] = l;
-      mbar_arrive(pair_bar);
-      if (warp_wait(pair_bar, static_cast<uint32_t>(nkv) & 1, abort_flag, tmo)) {
-        const float lt = __fadd_rn(xp[row], xp[kBM + row]);
-        tc_fence_after();
-        const int qrow = qt * kBM + row;
-        // O_acc ~ sum_k P8_k * code_k with P8 ~ 448 P~ and lt = sum 448 P~:
-        // O = RN(O_acc * v_scale) * RN(1 / lt) + v_mean (one fused multiply-add).
-        const float rl = __fdiv_rn(1.f, lt);
-        const int64_t obase = ((static_cast<int64_t>(b) * prm.N + qrow) * prm.H + h) * D + half * kOH;
-        const float* vf = s_vf + half * kOH;
-        const float* vm = s_vm + half * kOH;
+      tc_fence_after();
+      const int qrow = qt * kBM + row;
+      // O_acc ~ sum_k P8_k * code_k with P8 ~ 448 P~ and l = sum 448 P~:
+      // O = RN(O_acc * v_scale) * RN(1 / l) + v_mean (one fused multiply-add).
+      const float rl = __fdiv_rn(1.f, l);
+      const int64_t obase = ((static_cast<int64_t>(b) * prm.N + qrow) * prm.H + h) * D;
 #pragma unroll
-        for (int cb = 0; cb < kOH; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(to + cb, o);
-          tmem_wait_ld();
-          reg_fence(o);
-          float r[32];
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t o[32];
+        tmem_ld32(to + cb, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        float r[32];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 t = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
-                                   make_float2(vf[cb + i], vf[cb + i + 1]));
-            const float2 u = ffma2(t, make_float2(rl, rl), make_float2(vm[cb + i], vm[cb + i + 1]));
-            r[i] = u.x;
-            r[i + 1] = u.y;
-          }
-          if (qrow < prm.N) {
-            if (prm.out_fp32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + obase + cb);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 t = fmul2(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                 make_float2(s_vf[cb + i], s_vf[cb + i + 1]));
+          const float2 u = ffma2(t, make_float2(rl, rl), make_float2(s_vm[cb + i], s_vm[cb + i + 1]));
+          r[i] = u.x;
+          r[i + 1] = u.y;
+        }
+        if (qrow < prm.N) {
+          if (prm.out_fp32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.out) + obase + cb);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(prm.out) + obase + cb);
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(prm.out) + obase + cb);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t w[4];
+            for (int i = 0; i < 4; ++i) {
+              uint32_t w[4];
 #pragma unroll
-                for (int k2 = 0; k2 < 4; ++k2)
-                  w[k2] = float_to_bf16_bits(r[8 * i + 2 * k2]) | (float_to_bf16_bits(r[8 * i + 2 * k2 + 1]) << 16);
-                dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-              }
+              for (int k2 = 0; k2 < 4; ++k2)
+                w[k2] = float_to_bf16_bits(r[8 * i + 2 * k2]) | (float_to_bf16_bits(r[8 * i + 2 * k2 + 1]) << 16);
+              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
-        if (prm.lse && half == 0 && qrow < prm.N)
-          prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(lt) - kLog2P8) * 0.69314718055994531f;
       }
+      if (prm.lse && qrow < prm.N)
+        prm.lse[static_cast<int64_t>(bh) * prm.N + qrow] = (m + log2f(l) - kLog2P8) * 0.69314718055994531f;
     }
   }
 

@@ -320,6 +320,25 @@ __device__ __forceinline__ void tmem_ld64_pairs(uint32_t taddr, f32x2_t (&r)[32]
       : "r"(taddr)
       : "memory");
 }
+// 64 consecutive 32-bit columns of this warp's 32 lanes set to v: the value is
+// placed in one 8-register block once and stored 8 columns at a time (a 32-wide
+// store would need 32 registers holding it).  Await with tmem_wait_st().
+__device__ __forceinline__ void tmem_fill64(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "{.reg .b32 t0, t1, t2, t3, t4, t5, t6, t7;\n\t"
+      "mov.b32 t0, %1;\n\tmov.b32 t1, %1;\n\tmov.b32 t2, %1;\n\tmov.b32 t3, %1;\n\t"
+      "mov.b32 t4, %1;\n\tmov.b32 t5, %1;\n\tmov.b32 t6, %1;\n\tmov.b32 t7, %1;\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+8], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+16], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+24], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+32], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+40], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+48], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0+56], {t0, t1, t2, t3, t4, t5, t6, t7};\n\t"
+      "}" ::"r"(taddr), "r"(v)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // After tmem_wait_ld(): ties the loaded registers to this point, so that no use
 // of them is scheduled between the asynchronous tcgen05.ld and its wait.
@@ -449,6 +468,11 @@ __device__ __forceinline__ f32x2_t x2_fma(f32x2_t a, f32x2_t b, f32x2_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ f32x2_t x2_pack(uint32_t lo, uint32_t hi) {
+  f32x2_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
 __device__ __forceinline__ float x2_lo(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
 __device__ __forceinline__ float x2_hi(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 // Per 32-bit word: bits(p) + (bits(xr) << 23), i.e. the integer in the low bits
@@ -480,50 +504,53 @@ __device__ __forceinline__ uint32_t x2_e4m3x4(f32x2_t a, f32x2_t b) {
 // result is reproducible bit for bit on any IEEE machine (the CPU oracle runs
 // the same steps): Cody-Waite split x = n + f with n = round(x) by the
 // 1.5 * 2^23 addition (which leaves n, two's complement, in the low bits of
-// xr), f = x - n exactly, 2^f from a degree-5 polynomial with c0 = 1 fitted
-// for minimax relative error on [-1/2, 1/2] (linear programming; 2.2e-7 after
-// binary32 Horner evaluation with fused multiply-adds), and n added to the
-// exponent field of the polynomial's value: exactly p * 2^n for n >= -125.
+// xr), f = x - n exactly, 2^f from a polynomial with c0 = 1 fitted for minimax
+// relative error on [-1/2, 1/2] (linear programming), Horner with fused
+// multiply-adds, and n added to the exponent field of the polynomial's value:
+// exactly p * 2^n for n >= -125.  The per-key weights use a cubic (1.0e-4
+// relative after binary32 evaluation, far below the 6.25% step of the E4M3
+// codes they feed); the per-tile rescale factor a quintic (2.2e-7).
 // Requires x >= -126 (callers clamp).
 constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
-constexpr float kExp2C0 = 1.0f;
-constexpr float kExp2C1 = 0.6931465864181519f;
-constexpr float kExp2C2 = 0.24022166430950165f;
-constexpr float kExp2C3 = 0.055510472506284714f;
-constexpr float kExp2C4 = 0.009674952365458012f;
-constexpr float kExp2C5 = 0.0013202981790527701f;
+constexpr float kExp2C1 = 0.6932829022407532f;   // cubic
+constexpr float kExp2C2 = 0.2422109693288803f;
+constexpr float kExp2C3 = 0.055009059607982635f;
+constexpr float kExp2Q1 = 0.6931465864181519f;   // quintic
+constexpr float kExp2Q2 = 0.24022166430950165f;
+constexpr float kExp2Q3 = 0.055510472506284714f;
+constexpr float kExp2Q4 = 0.009674952365458012f;
+constexpr float kExp2Q5 = 0.0013202981790527701f;
 constexpr float kExp2Min = -126.0f;
 
 // The constant pairs of exp2_fixed_x2, built once per thread.
 struct Exp2Consts {
-  f32x2_t round, c0, c1, c2, c3, c4, c5;
+  f32x2_t round, c0, c1, c2, c3;
   __device__ __forceinline__ Exp2Consts()
-      : round(x2_splat(kExp2Round)), c0(x2_splat(kExp2C0)), c1(x2_splat(kExp2C1)), c2(x2_splat(kExp2C2)),
-        c3(x2_splat(kExp2C3)), c4(x2_splat(kExp2C4)), c5(x2_splat(kExp2C5)) {}
+      : round(x2_splat(kExp2Round)), c0(x2_splat(1.0f)), c1(x2_splat(kExp2C1)), c2(x2_splat(kExp2C2)),
+        c3(x2_splat(kExp2C3)) {}
 };
 
+// Cubic form on a pair.
 __device__ __forceinline__ f32x2_t exp2_fixed_x2(f32x2_t x, const Exp2Consts& k) {
   const f32x2_t xr = x2_add(x, k.round);
   const f32x2_t nf = x2_sub(xr, k.round);
   const f32x2_t f = x2_sub(x, nf);
-  f32x2_t p = x2_fma(k.c5, f, k.c4);
-  p = x2_fma(p, f, k.c3);
-  p = x2_fma(p, f, k.c2);
+  f32x2_t p = x2_fma(k.c3, f, k.c2);
   p = x2_fma(p, f, k.c1);
   p = x2_fma(p, f, k.c0);
   return x2_add_exponent(p, xr);
 }
-// Scalar form, clamping x at -126 itself.
-__device__ __forceinline__ float exp2_fixed(float x) {
+// Quintic scalar form, clamping x at -126 itself.
+__device__ __forceinline__ float exp2_fixed5(float x) {
   x = fmaxf(x, kExp2Min);
   const float xr = __fadd_rn(x, kExp2Round);
   const float nf = __fadd_rn(xr, -kExp2Round);
   const float f = __fsub_rn(x, nf);
-  float p = __fmaf_rn(kExp2C5, f, kExp2C4);
-  p = __fmaf_rn(p, f, kExp2C3);
-  p = __fmaf_rn(p, f, kExp2C2);
-  p = __fmaf_rn(p, f, kExp2C1);
-  p = __fmaf_rn(p, f, kExp2C0);
+  float p = __fmaf_rn(kExp2Q5, f, kExp2Q4);
+  p = __fmaf_rn(p, f, kExp2Q3);
+  p = __fmaf_rn(p, f, kExp2Q2);
+  p = __fmaf_rn(p, f, kExp2Q1);
+  p = __fmaf_rn(p, f, 1.0f);
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(xr) << 23));
 }
 

@@ -212,25 +212,30 @@ def quant_v(v_bits: np.ndarray):
 # ----------------------------------------------------------------------------
 # exp2 of the FP32 softmax (reading: the pages fix FP32 for the softmax but not
 # how exp2 is evaluated; this contract fixes it so that every P8 code is
-# reproducible).  Cody-Waite split with round-to-nearest, then a degree-5
-# polynomial with c0 = 1 fitted for minimax relative error on [-1/2, 1/2]
-# (oracle/fit_exp2.py; 2.2e-7 after binary32 evaluation), then n added to the
-# exponent field.
-EXP2_C = tuple(np.float32(v) for v in (1.0, 0.6931465864181519, 0.24022166430950165,
-                                       0.055510472506284714, 0.009674952365458012,
-                                       0.0013202981790527701))
+# reproducible).  Cody-Waite split with round-to-nearest, then a polynomial
+# with c0 = 1 fitted for minimax relative error on [-1/2, 1/2]
+# (oracle/fit_exp2.py), then n added to the exponent field.  The per-key
+# weights use a cubic (1.0e-4 after binary32 evaluation, 600 times below the
+# 6.25% relative step of the E4M3 codes they feed); the once-per-tile rescale
+# factor, whose error would compound over tiles in the row sum, a quintic
+# (2.2e-7).
+EXP2_C = tuple(np.float32(v) for v in (1.0, 0.6932829022407532, 0.2422109693288803,
+                                       0.055009059607982635))
+EXP2_C5 = tuple(np.float32(v) for v in (1.0, 0.6931465864181519, 0.24022166430950165,
+                                        0.055510472506284714, 0.009674952365458012,
+                                        0.0013202981790527701))
 EXP2_MIN = np.float32(-126.0)
 EXP2_ROUND = np.float32(12582912.0)   # 1.5 * 2^23
 
 
-def exp2_contract(u) -> np.ndarray:
+def exp2_contract(u, coeffs=EXP2_C) -> np.ndarray:
     """2^u as the contract evaluates it, every step a binary32 operation.
 
       x  = max(u, -126)
       xr = RN(x + 1.5 * 2^23)           the integer n = round(x) in the low bits (two's complement)
       nf = RN(xr - 1.5 * 2^23)          = n, exactly
       f  = RN(x - nf)                   exact, |f| <= 1/2
-      p  = c5; p = fma(p, f, c_k) for k = 4 .. 0
+      p  = c_d; p = fma(p, f, c_k) for k = d - 1 .. 0 (coeffs = c_0 .. c_d)
       y  = the binary32 whose bits are bits(p) + (bits(xr) << 23) mod 2^32,
            i.e. n added to the exponent field of p: exactly p * 2^n for
            n >= -125 (p lies in [2^-1/2, 2^1/2]); at n = -126 a value below
@@ -240,18 +245,22 @@ def exp2_contract(u) -> np.ndarray:
     xr = rn32(x.astype(np.float64) + np.float64(EXP2_ROUND))
     nf = rn32(xr.astype(np.float64) - np.float64(EXP2_ROUND))
     f = rn32(x.astype(np.float64) - nf.astype(np.float64))
-    p = np.full(f.shape, EXP2_C[5], dtype=np.float32)
-    for k in (4, 3, 2, 1, 0):
-        p = fma32(p, f, EXP2_C[k])
+    p = np.full(f.shape, coeffs[-1], dtype=np.float32)
+    for ck in coeffs[-2::-1]:
+        p = fma32(p, f, ck)
     bits = p.view(np.uint32) + (xr.view(np.uint32) << np.uint32(23))   # uint32 arithmetic wraps
     return bits.astype(np.uint32).view(np.float32)
+
+
+def _exp2_alpha(x):
+    return exp2_contract(x, EXP2_C5)
 
 
 def _identity(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, quant_p,
+def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2_alpha, quant_p,
                  log2_p_unit, two_pass=False):
     """Online-softmax attention over 128-key tiles for one (b, h).
 
@@ -264,7 +273,8 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, quan
               mean added back.
     rn        rounding applied after every step (rn32, or identity in FP64).
     fma       fused multiply-add with one rounding (fma32, or exact in FP64).
-    exp2      the exp2 of the softmax (exp2_contract, or np.exp2 in FP64).
+    exp2      the exp2 of the per-key weights (exp2_contract, or np.exp2 in FP64);
+    exp2_alpha  the exp2 of the rescale factor (exp2_contract with the quintic).
     quant_p   P quantizer (E4M3 round trip, or identity).
     log2_p_unit  log2 of the P scale folded into the exponent: RN32(log2 448)
               with quantization on, 0 with it off.
@@ -272,7 +282,7 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, quan
     Per tile j (keys j0..j1-1, those >= n_keys excluded):
       t     = rn(S * c)                          scores in the exp2 domain
       m_new = max(m, max_k t)                    running row max
-      alpha = exp2(rn(m - m_new))                (~0 on the first tile, m = -inf)
+      alpha = exp2_alpha(rn(m - m_new))          (0 on the first tile, m = -inf)
       e     = rn(log2_p_unit - m_new)
       y     = exp2(fma(S, c, e))                 = P~ * 448, P~ = exp2(t - m_new)
       l     = rn(rn(l * alpha) + rn(sum_k y))    row sum of the unquantized y
@@ -300,7 +310,7 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, quan
         t = rn(S[:, j0:j1] * c)
         m_new = m if two_pass else np.maximum(m, t.max(axis=1))
         with np.errstate(invalid="ignore"):
-            alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2(rn(m - m_new)), dtype=np.float64))
+            alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2_alpha(rn(m - m_new)), dtype=np.float64))
         if two_pass:
             alpha = np.ones(R)
         e = rn(log2_p_unit - m_new)
@@ -370,7 +380,7 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
         Vt = e4m3_decode(v_codes_t[b, h, :, :N])
         o, m, l = _attend_rows(S, col_mult, Vt, v_scale[b, h].astype(np.float64),
                                v_mean[b, h].astype(np.float64), N, rn32, fma32, exp2_contract,
-                               _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass)
+                               _exp2_alpha, _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass)
         out[b, :, h, :] = o
         lse[b, h] = rn32((m + np.log2(l) - math.log2(E4M3_MAX)) * math.log(2.0))
     return (out, lse) if want_lse else out
@@ -402,7 +412,7 @@ def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
         mean = V.mean(axis=0) if smooth_v else np.zeros(D)
         S = Q @ K.T
         o, _, _ = _attend_rows(S, lambda j0, j1: c, (V - mean).T, np.ones(D), mean,
-                               N, _identity, _fma_exact, np.exp2, _identity, 0.0)
+                               N, _identity, _fma_exact, np.exp2, np.exp2, _identity, 0.0)
         out[b, :, h, :] = o
     return out
 
