@@ -93,6 +93,30 @@ def quant_bytes(w):
     return qk, v
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_env():
+    """(rank, world size, local rank) of this process, as torchrun sets them."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (every rank gets it); x itself when alone."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(world: int, ops_per_step: float, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of its own batch
+    (replicas), so the job does world * ops * steps in the slowest rank's time."""
+    return world * ops_per_step * steps / (max_total_ms / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -202,9 +226,7 @@ def run_reference(args, rank):
 # ----------------------------------------------------------------------------- ours
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     if args.impl == "reference":
         run_reference(args, rank)
         return
@@ -274,13 +296,9 @@ def main():
     qk_ms = [e[0].elapsed_time(e[1]) for e in ev]
     v_ms = [e[1].elapsed_time(e[2]) for e in ev]
     at_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     ops = w.attn_ops
-    value = world * ops * K / (max_total_ms / 1e3) / 1e12
+    value = job_tops(world, ops, K, max_total_ms)
 
     # --------------------------------------------------------------- e2e (host buffers)
     pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
@@ -303,11 +321,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     adt.sage_check()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * ops * K / (float(t.item()) / 1e3) / 1e12
+    e2e_value = job_tops(world, ops, K, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, "cuda"))
     h2d = 3 * qb.nbytes
     d2h = buf.out.numel() * buf.out.element_size()
 
