@@ -333,7 +333,9 @@ def main():
     qk_bytes, v_bytes = quant_bytes(w)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows, heads = 512, 2
+        # about 10-30 s of CPU work on the GPU machine's host: 4 heads, 2^26 (query row, key) pairs
+        heads = min(4, w.H)
+        rows = max(1, min(w.N, (1 << 26) // (heads * w.N)))
         o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads)
         cpu = {"value": o_ops / o_dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{heads} heads of batch 0: full K/V quantization of those heads + attention for "
