@@ -106,27 +106,51 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
 template <bool kMasked, bool kClamp>
 __device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], f32x2_t c2, f32x2_t e2, int valid,
                                                 const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
-  f32x2_t prev = 0;
+  // Stage-major over 8 pairs at a time: every step is issued for 8 independent
+  // pairs before the next step, so consecutive instructions do not depend on
+  // each other.
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const f32x2_t sv = x2_sub(x2_pack(s[2 * i], s[2 * i + 1]), k.round);  // exact integer S (the S bias is 1.5 * 2^23 too)
-    f32x2_t u = x2_fma(sv, c2, e2);
+  for (int h8 = 0; h8 < 2; ++h8) {
+    f32x2_t u[8], xr[8], f[8], p[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * h8 + i;
+      u[i] = x2_sub(x2_pack(s[2 * j], s[2 * j + 1]), k.round);   // exact integer S (the S bias is 1.5 * 2^23 too)
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = x2_fma(u[i], c2, e2);
     if (kClamp) {
-      const float lo = fmaxf(x2_lo(u), kExp2Min);
-      const float hi = fmaxf(x2_hi(u), kExp2Min);
-      u = (static_cast<f32x2_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        u[i] = x2_pack(__float_as_uint(fmaxf(x2_lo(u[i]), kExp2Min)), __float_as_uint(fmaxf(x2_hi(u[i]), kExp2Min)));
     }
-    f32x2_t y = exp2_fixed_x2(u, k);
-    if (kMasked) {
-      const uint32_t lo = 2 * i < valid ? static_cast<uint32_t>(y) : 0u;
-      const uint32_t hi = 2 * i + 1 < valid ? static_cast<uint32_t>(y >> 32) : 0u;
-      y = (static_cast<f32x2_t>(hi) << 32) | lo;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) xr[i] = x2_add(u[i], k.round);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = x2_sub(xr[i], k.round);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = x2_sub(u[i], f[i]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = x2_fma(k.c3, f[i], k.c2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f32x2_t y = x2_add_exponent(p[i], xr[i]);
+      if (kMasked) {
+        const int j = 8 * h8 + i;
+        const uint32_t lo = 2 * j < valid ? static_cast<uint32_t>(y) : 0u;
+        const uint32_t hi = 2 * j + 1 < valid ? static_cast<uint32_t>(y >> 32) : 0u;
+        y = (static_cast<f32x2_t>(hi) << 32) | lo;
+      }
+      p[i] = y;
     }
-    lsum[i & 3] = x2_add(lsum[i & 3], y);              // four independent partial sums
-    if (i & 1)
-      pk[i >> 1] = x2_e4m3x4(prev, y);
-    else
-      prev = y;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) lsum[i & 3] = x2_add(lsum[i & 3], p[i]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pk[4 * h8 + i] = x2_e4m3x4(p[2 * i], p[2 * i + 1]);
   }
 }
 
