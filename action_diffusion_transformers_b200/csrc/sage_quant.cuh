@@ -81,12 +81,12 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
     }
   };
   int n = n0;
-  for (; n + 8 <= n1; n += 8) {
-    uint4 raw[8];
+  for (; n + 16 <= n1; n += 16) {         // 16 loads in flight
+    uint4 raw[16];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) raw[t] = ld_nc_16(p + static_cast<int64_t>(n - n0 + t) * tok_stride);
+    for (int t = 0; t < 16; ++t) raw[t] = ld_nc_16(p + static_cast<int64_t>(n - n0 + t) * tok_stride);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) accumulate(raw[t]);
+    for (int t = 0; t < 16; ++t) accumulate(raw[t]);
   }
   for (; n < n1; ++n) accumulate(ld_nc_16(p + static_cast<int64_t>(n - n0) * tok_stride));
   const int64_t o = (static_cast<int64_t>(b) * nsb + c) * HD + ch0;
