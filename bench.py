@@ -80,6 +80,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="action_dit", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--peaks", action="store_true",
+                    help="measure library INT8 / FP8 / BF16 GEMM throughput at 8192^3 and exit")
     return ap.parse_args()
 
 
@@ -223,10 +225,49 @@ def run_reference(args, rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- peaks
+def measure_peaks(reps: int = 20):
+    """Dense GEMM throughput of the libraries torch calls (cuBLAS / cuBLASLt) at
+    8192^3: torch._int_mm (INT8 -> INT32), torch._scaled_mm (FP8 E4M3 -> BF16)
+    and torch.matmul (BF16), best of `reps` event-timed calls.  Context for the
+    attention roofline, whose peak stays the measured BF16 figure x 2."""
+    import torch
+    n = 8192
+    torch.manual_seed(0)
+    a8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda")
+    b8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device="cuda").t()
+    af = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+    bf = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device="cuda")
+    ab = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+    bb = torch.randn(n, n, device="cuda", dtype=torch.bfloat16)
+    cases = {"int8_tops": lambda: torch._int_mm(a8, b8),
+             "fp8_tflops": lambda: torch._scaled_mm(af, bf, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+             "bf16_tflops": lambda: ab @ bb}
+    out = {}
+    for name, fn in cases.items():
+        for _ in range(3):
+            fn()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out[name] = 2.0 * n ** 3 / (best / 1e3) / 1e12
+    return out
+
+
 # ----------------------------------------------------------------------------- ours
 def main():
     args = parse()
     rank, world, local = rank_env()
+    if args.peaks:
+        if rank == 0:
+            print(json.dumps({"peaks": measure_peaks(), "shape": "8192^3", "best_of": 20}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, rank)
         return
