@@ -80,10 +80,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
-// Named barrier `id` over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
@@ -193,34 +189,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 #undef SAGE_R8
-#define SAGE_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
-                   "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      SAGE_W8(0), SAGE_W8(8), SAGE_W8(16), SAGE_W8(24)
-      : "memory");
-}
-#undef SAGE_W8
-// 16 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-// 32 consecutive TMEM columns of this thread's lane all set to `v`.
-__device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,"
-      "%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr), "r"(v)
-      : "memory");
-}
 // 32 consecutive 32-bit columns, waited for and returned as 16 pairs.
 __device__ __forceinline__ void tmem_ld32_pairs(uint32_t taddr, f32x2_t (&r)[16]) {
   asm volatile(
@@ -273,51 +241,6 @@ __device__ __forceinline__ void tmem_st32_pairs(uint32_t taddr, const f32x2_t (&
       "}"
       :
       : "r"(taddr), "l"(r[0]), "l"(r[1]), "l"(r[2]), "l"(r[3]), "l"(r[4]), "l"(r[5]), "l"(r[6]), "l"(r[7]), "l"(r[8]), "l"(r[9]), "l"(r[10]), "l"(r[11]), "l"(r[12]), "l"(r[13]), "l"(r[14]), "l"(r[15])
-      : "memory");
-}
-// 64 consecutive 32-bit columns of this warp's 32 TMEM lanes, waited for and
-// returned as 32 pairs (column 2i in the low word of r[i]).  The wait is inside
-// the same asm statement, so the pairs are never read before the load lands.
-__device__ __forceinline__ void tmem_ld64_pairs(uint32_t taddr, f32x2_t (&r)[32]) {
-  asm volatile(
-      "{.reg .b32 t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31, t32, t33, t34, t35, t36, t37, t38, t39, t40, t41, t42, t43, t44, t45, t46, t47, t48, t49, t50, t51, t52, t53, t54, t55, t56, t57, t58, t59, t60, t61, t62, t63;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {t0, t1, t2, t3, t4, t5, t6, t7, t8, t9, t10, t11, t12, t13, t14, t15, t16, t17, t18, t19, t20, t21, t22, t23, t24, t25, t26, t27, t28, t29, t30, t31, t32, t33, t34, t35, t36, t37, t38, t39, t40, t41, t42, t43, t44, t45, t46, t47, t48, t49, t50, t51, t52, t53, t54, t55, t56, t57, t58, t59, t60, t61, t62, t63}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;\n\t"
-      "mov.b64 %0, {t0, t1};\n\t"
-      "mov.b64 %1, {t2, t3};\n\t"
-      "mov.b64 %2, {t4, t5};\n\t"
-      "mov.b64 %3, {t6, t7};\n\t"
-      "mov.b64 %4, {t8, t9};\n\t"
-      "mov.b64 %5, {t10, t11};\n\t"
-      "mov.b64 %6, {t12, t13};\n\t"
-      "mov.b64 %7, {t14, t15};\n\t"
-      "mov.b64 %8, {t16, t17};\n\t"
-      "mov.b64 %9, {t18, t19};\n\t"
-      "mov.b64 %10, {t20, t21};\n\t"
-      "mov.b64 %11, {t22, t23};\n\t"
-      "mov.b64 %12, {t24, t25};\n\t"
-      "mov.b64 %13, {t26, t27};\n\t"
-      "mov.b64 %14, {t28, t29};\n\t"
-      "mov.b64 %15, {t30, t31};\n\t"
-      "mov.b64 %16, {t32, t33};\n\t"
-      "mov.b64 %17, {t34, t35};\n\t"
-      "mov.b64 %18, {t36, t37};\n\t"
-      "mov.b64 %19, {t38, t39};\n\t"
-      "mov.b64 %20, {t40, t41};\n\t"
-      "mov.b64 %21, {t42, t43};\n\t"
-      "mov.b64 %22, {t44, t45};\n\t"
-      "mov.b64 %23, {t46, t47};\n\t"
-      "mov.b64 %24, {t48, t49};\n\t"
-      "mov.b64 %25, {t50, t51};\n\t"
-      "mov.b64 %26, {t52, t53};\n\t"
-      "mov.b64 %27, {t54, t55};\n\t"
-      "mov.b64 %28, {t56, t57};\n\t"
-      "mov.b64 %29, {t58, t59};\n\t"
-      "mov.b64 %30, {t60, t61};\n\t"
-      "mov.b64 %31, {t62, t63};\n\t"
-      "}"
-      : "=l"(r[0]), "=l"(r[1]), "=l"(r[2]), "=l"(r[3]), "=l"(r[4]), "=l"(r[5]), "=l"(r[6]), "=l"(r[7]), "=l"(r[8]), "=l"(r[9]), "=l"(r[10]), "=l"(r[11]), "=l"(r[12]), "=l"(r[13]), "=l"(r[14]), "=l"(r[15]), "=l"(r[16]), "=l"(r[17]), "=l"(r[18]), "=l"(r[19]), "=l"(r[20]), "=l"(r[21]), "=l"(r[22]), "=l"(r[23]), "=l"(r[24]), "=l"(r[25]), "=l"(r[26]), "=l"(r[27]), "=l"(r[28]), "=l"(r[29]), "=l"(r[30]), "=l"(r[31])
-      : "r"(taddr)
       : "memory");
 }
 // 64 consecutive 32-bit columns of this warp's 32 lanes set to v: the value is
@@ -401,17 +324,6 @@ __device__ __forceinline__ uint32_t double_to_bf16_bits(double x) {
   return sign | bits;
 }
 
-// ---------------------------------------------------------------- packed FP32
-// Two-lane FP32 arithmetic (sm_100 f32x2 instructions): one issue slot for two
-// results.  Each rounds like its scalar counterpart.
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   float2 d;
   asm("{.reg .b64 ra, rb, rd;\n\t"

@@ -10,7 +10,9 @@ the oracle computes head by head and row by row:
   long-video workload, whose Student-t(3) rows make a few softmax rows hinge
   on large INT8 scores: there the method itself (the oracle, and equally a
   per-token INT8 variant) reaches about 0.998, so the check is >= 0.997;
-* the BF16 output equals the RNE rounding of the FP32 output on those rows.
+* the BF16 output equals the RNE rounding of the FP32 output on those rows;
+* the LSE of those rows within 1e-4 (relative to max(1, |lse|)) of the oracle's.
+A D = 64 shape with many KV tiles and a ragged tail runs the same checks.
 """
 import numpy as np
 import pytest
@@ -42,16 +44,20 @@ def _cos(a, b):
     return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
 
 
-@pytest.mark.parametrize("name", ["action_dit", "mid_video", "long_video", "ragged"])
+@pytest.mark.parametrize("name", ["action_dit", "mid_video", "long_video", "ragged", "d64_many_tiles"])
 def test_full_size_sampled_parity(adt, name):
-    w = synth.WORKLOADS[name]
+    if name == "d64_many_tiles":
+        w = synth.custom(1, 8200, 8, 64, seed=7, k_sigma=4.0, v_sigma=1.0, outlier_frac=0.02)
+    else:
+        w = synth.WORKLOADS[name]
     qb, kb, vb = synth.generate(w)
     q, k, v = _dev(qb), _dev(kb), _dev(vb)
     buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens)
     out16 = buf.run(q, k, v)
     out32 = torch.empty((w.B, w.N, w.H, w.D), dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
     adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
-                      buf.v_mean, buf.shape, 0.0, out32, True)
+                      buf.v_mean, buf.shape, 0.0, out32, True, lse)
     adt.sage_check()
 
     heads = [(0, 0), (w.B - 1, w.H - 1), (0, w.H // 2)]
@@ -72,8 +78,13 @@ def test_full_size_sampled_parity(adt, name):
         assert np.array_equal(got(buf.v_mean).view(np.uint32), ref_v["v_mean"].view(np.uint32))
         if i >= 2:
             continue
-        ref = so.attn_fwd(ref_qk["q_codes"], ref_qk["q_scale"], ref_qk["k_codes"], ref_qk["k_scale"],
-                          ref_v["v_codes_t"], ref_v["v_scale"], ref_v["v_mean"], w.N, rows=rows)[0, :, 0, :]
+        ref, ref_lse = so.attn_fwd(ref_qk["q_codes"], ref_qk["q_scale"], ref_qk["k_codes"], ref_qk["k_scale"],
+                                   ref_v["v_codes_t"], ref_v["v_scale"], ref_v["v_mean"], w.N, rows=rows,
+                                   want_lse=True)
+        ref = ref[0, :, 0, :]
+        ref_lse = ref_lse[0, 0]
+        got_lse = lse[b, h, rows].cpu().numpy()
+        assert np.abs(got_lse - ref_lse).max() <= 1e-4 * max(1.0, np.abs(ref_lse).max())
         g32 = out32[b, rows, h, :].cpu().numpy()
         assert np.all(np.isfinite(g32))
         err = np.abs(g32 - ref).max()
