@@ -24,8 +24,9 @@ floating-point step that the GPU does in FP32 is rounded to FP32 here
 (``rn32``); exact integer dot products are formed in float64, which is exact
 for |sum| < 2**53.
 
-Parity status: pinned by tests/test_oracle_sage.py (quantizers by brute force
-and invariants; the attention tile loop by running it with quantization off
+Parity status: pinned by tests/test_oracle_sage.py and
+tests/test_oracle_granularity.py (quantizers by brute force and invariants at
+every scale granularity: 64-token blocks, per token, segment-local blocks; the attention tile loop by running it with quantization off
 against brute-force FP64 softmax attention; smoothing by the softmax shift
 invariance; closed forms for degenerate inputs; the softmax exp2 against
 numpy's exp2 within its stated error bound and exactly at integers; the fused
@@ -100,27 +101,88 @@ def column_sum_f64(x: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 # A2: INT8 block quantization (Q as is, K after centring)
 # ----------------------------------------------------------------------------
-def int8_block_quant(x: np.ndarray):
-    """Quantize x[B, H, Npad, D] (float32, zero in padded rows) per 64-token block.
+GRANULARITIES = ("block64", "token", "segment64")
 
-    For each (b, h, block of 64 consecutive tokens, all D channels):
-      amax  = max |x| over the block,
+
+def scale_groups(N: int, gran: str = "block64", cu_seqlens=None) -> np.ndarray:
+    """First token of every INT8 scale group on the padded token axis [0, Npad).
+
+    Groups are runs of consecutive tokens; every group spans all D channels.
+      block64    64-token blocks on one grid over the whole sequence (the
+                 configurations' "Q/K INT8 blocks 64 tokens");
+      token      one group per token (the tcgen05 counterpart of the pages'
+                 per-thread granularity, which gives each GPU thread its own
+                 scale: here one thread owns one query row);
+      segment64  64-token blocks restarting at every segment start of a packed
+                 joint sequence (cu_seqlens), so that no block mixes two streams;
+                 the last block of a segment may be short.
+    Padded tokens [N, Npad) hold zeros; in segment64 they form blocks of their
+    own, on the 64-token grid that continues from N.
+    """
+    Np = npad(N)
+    if gran == "block64":
+        return np.arange(0, Np, QK_BLOCK)
+    if gran == "token":
+        return np.arange(Np)
+    if gran == "segment64":
+        cu = [0, N] if cu_seqlens is None else [int(c) for c in cu_seqlens]
+        starts = []
+        for a, e in zip(cu[:-1], cu[1:]):
+            starts.extend(range(a, e, QK_BLOCK))
+        starts.extend(range(N, Np, QK_BLOCK))
+        return np.asarray(starts, dtype=np.int64)
+    raise ValueError(f"unknown granularity {gran!r}")
+
+
+def int8_group_quant(x: np.ndarray, starts: np.ndarray):
+    """Quantize x[B, H, Npad, D] (float32, zero in padded rows) per scale group.
+
+    starts: first token of each group (increasing, starts[0] == 0); group g is
+    tokens [starts[g], starts[g+1]) over all D channels.  For each (b, h, group):
+      amax  = max |x| over the group,
       scale = RN32(amax / 127),  inv = RN32(127 / amax),
       code  = clamp(RNE(RN32(x * inv)), -127, 127);
     amax == 0 gives scale = inv = 0 and all codes 0.
-    Returns (codes int8 [B, H, Npad, D], scale float32 [B, H, Npad/64]).
+    Returns (codes int8 [B, H, Npad, D], scale float32 [B, H, n_groups]).
     """
     x = np.asarray(x, dtype=np.float32)
     B, H, Np, D = x.shape
-    xb = x.reshape(B, H, Np // QK_BLOCK, QK_BLOCK, D)
-    amax = np.max(np.abs(xb), axis=(3, 4))
+    starts = np.asarray(starts, dtype=np.int64)
+    lengths = np.diff(np.append(starts, Np))
+    amax = np.maximum.reduceat(np.abs(x).max(axis=3), starts, axis=2)     # [B, H, G]
     nz = amax > 0
     safe = np.where(nz, amax, np.float32(1))
     scale = np.where(nz, safe / np.float32(INT8_MAX), np.float32(0)).astype(np.float32)
     inv = np.where(nz, np.float32(INT8_MAX) / safe, np.float32(0)).astype(np.float32)
-    prod = (xb * inv[..., None, None]).astype(np.float32)
+    inv_tok = np.repeat(inv, lengths, axis=2)                              # [B, H, Npad]
+    prod = (x * inv_tok[..., None]).astype(np.float32)
     codes = np.clip(np.rint(prod), -INT8_MAX, INT8_MAX).astype(np.int8)
-    return codes.reshape(B, H, Np, D), scale
+    return codes, scale
+
+
+def int8_block_quant(x: np.ndarray):
+    """int8_group_quant on 64-token blocks: (codes [B, H, Npad, D], scale [B, H, Npad/64])."""
+    return int8_group_quant(x, np.arange(0, x.shape[2], QK_BLOCK))
+
+
+def quant_scales(x: np.ndarray, N: int, gran: str = "block64", cu_seqlens=None):
+    """INT8 codes and scales of x[B, H, Npad, D] at a granularity, in the layout
+    the attention call reads: block64 -> scale [B, H, Npad/64] (one per block);
+    token, segment64 -> scale [B, H, Npad] (every token holds its group's scale)."""
+    starts = scale_groups(N, gran, cu_seqlens)
+    codes, scale = int8_group_quant(x, starts)
+    if gran == "block64":
+        return codes, scale
+    lengths = np.diff(np.append(starts, x.shape[2]))
+    return codes, np.repeat(scale, lengths, axis=2)
+
+
+def token_scales(scale: np.ndarray, Np: int) -> np.ndarray:
+    """The per-token view of a Q or K scale array in either layout."""
+    if scale.shape[-1] == Np:
+        return scale
+    assert scale.shape[-1] * QK_BLOCK == Np, scale.shape
+    return np.repeat(scale, QK_BLOCK, axis=-1)
 
 
 def _nhd_to_bhnd_padded(x32: np.ndarray) -> np.ndarray:
@@ -142,23 +204,26 @@ def k_mean_bf16(k_bits: np.ndarray) -> np.ndarray:
     return f64_to_bf16_bits(s / np.float64(N)).reshape(B, H, D)
 
 
-def quant_qk(q_bits: np.ndarray, k_bits: np.ndarray):
-    """A1-A3: K smoothing and INT8 block quantization of Q and K.
+def quant_qk(q_bits: np.ndarray, k_bits: np.ndarray, q_gran: str = "block64",
+             k_gran: str = "block64", cu_seqlens=None):
+    """A1-A3: K smoothing and INT8 quantization of Q and K.
 
     q_bits, k_bits: BF16 bit patterns uint16 [B, N, H, D].
-    K is centred by its BF16 token mean and rounded back to BF16 before
-    quantization:  kc = RN_bf16(RN32(k - mean_k)).  Q is quantized raw (the
-    pages keep only K and V smoothing).
+    K is centred by its BF16 token mean (over all N tokens, whatever the scale
+    granularity) and rounded back to BF16 before quantization:
+    kc = RN_bf16(RN32(k - mean_k)).  Q is quantized raw (the pages keep only K
+    and V smoothing).  q_gran / k_gran pick the scale groups (scale_groups).
     Returns dict with q_codes, q_scale, k_codes, k_scale (layouts as
-    int8_block_quant) and k_mean (uint16 [B, H, D]).
+    quant_scales) and k_mean (uint16 [B, H, D]).
     """
+    N = q_bits.shape[1]
     q32 = bf16_bits_to_f32(q_bits)
     k32 = bf16_bits_to_f32(k_bits)
     mean_bits = k_mean_bf16(k_bits)
     mean32 = bf16_bits_to_f32(mean_bits)                       # [B, H, D]
     kc = round_f32_to_bf16((k32 - mean32[:, None, :, :]).astype(np.float32))
-    q_codes, q_scale = int8_block_quant(_nhd_to_bhnd_padded(q32))
-    k_codes, k_scale = int8_block_quant(_nhd_to_bhnd_padded(kc))
+    q_codes, q_scale = quant_scales(_nhd_to_bhnd_padded(q32), N, q_gran, cu_seqlens)
+    k_codes, k_scale = quant_scales(_nhd_to_bhnd_padded(kc), N, k_gran, cu_seqlens)
     return dict(q_codes=q_codes, q_scale=q_scale, k_codes=k_codes,
                 k_scale=k_scale, k_mean=mean_bits)
 
@@ -345,10 +410,12 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
              sm_scale=None, rows=None, heads=None, two_pass=False, want_lse=False):
     """A6-A10 on quantized operands; the output is the FP32 attention output.
 
-    q_codes, k_codes int8 [B, H, Npad, D]; q_scale, k_scale f32 [B, H, Npad/64];
+    q_codes, k_codes int8 [B, H, Npad, D]; q_scale, k_scale f32 [B, H, Npad/64]
+    (one per 64-token block) or [B, H, Npad] (one per token, see quant_scales);
     v_codes_t uint8 E4M3 [B, H, D, Npad]; v_scale, v_mean f32 [B, H, D].
-    Score dequant multiplier for query row i and key j:
-        c = RN32(RN32(qs[i // 64] * ks[j // 64]) * RN32(sm_scale * log2 e)),
+    Score dequant multiplier for query row i and key j, with qs[i] and ks[j]
+    the scales of the groups that hold token i of Q and token j of K:
+        c = RN32(RN32(qs[i] * ks[j]) * RN32(sm_scale * log2 e)),
     the P scale 448 enters the exponent as RN32(log2 448) (P8 = E4M3(P~ * 448),
     with the exponent of P~ * 448 formed by one fused multiply-add), the row
     sum holds P~ * 448 and the output factor is the V scale itself.
@@ -370,11 +437,11 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
         Qf = q_codes[b, h, rows].astype(np.float64)
         Kf = k_codes[b, h, :N].astype(np.float64)
         S = Qf @ Kf.T                                        # exact INT32 dots
-        qs = q_scale[b, h, rows // QK_BLOCK]
-        ks = k_scale[b, h]
+        qs = token_scales(q_scale[b, h], Np)[rows]
+        ks = token_scales(k_scale[b, h], Np)
 
         def col_mult(j0, j1, qs=qs, ks=ks):
-            kk = ks[np.arange(j0, j1) // QK_BLOCK]
+            kk = ks[j0:j1]
             return rn32(rn32(qs[:, None].astype(np.float64) * kk[None, :]) * np.float64(sl2e))
 
         Vt = e4m3_decode(v_codes_t[b, h, :, :N])
@@ -437,10 +504,10 @@ def attn_exact_fp64(q, k, v, N, sm_scale=None, rows=None, heads=None):
 
 
 def sage_pipeline(q_bits, k_bits, v_bits, sm_scale=None, rows=None, heads=None,
-                  two_pass=False):
+                  two_pass=False, q_gran="block64", k_gran="block64", cu_seqlens=None):
     """Whole path A1-A10 from BF16 inputs: returns (fp32 output, intermediates)."""
     N = q_bits.shape[1]
-    qk = quant_qk(q_bits, k_bits)
+    qk = quant_qk(q_bits, k_bits, q_gran, k_gran, cu_seqlens)
     vv = quant_v(v_bits)
     o = attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"],
                  vv["v_codes_t"], vv["v_scale"], vv["v_mean"], N, sm_scale=sm_scale,
