@@ -35,10 +35,14 @@ EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v"
 QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
+GRAN = {"block64": 0, "token": 1, "segment64": 2}   # sage_gran: INT8 scale groups of Q / K
+MAX_SEGMENTS = 256
+
+
 class SageShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("H", ctypes.c_int), ("D", ctypes.c_int),
                 ("tok_stride", ctypes.c_int64), ("cu_seqlens", ctypes.POINTER(ctypes.c_int32)),
-                ("n_seg", ctypes.c_int)]
+                ("n_seg", ctypes.c_int), ("q_gran", ctypes.c_int), ("k_gran", ctypes.c_int)]
 
 
 _vp = ctypes.c_void_p
@@ -77,8 +81,9 @@ def _ok(status: int, where: str) -> None:
         raise SageError(status, where)
 
 
-def make_shape(B, N, H, D, tok_stride=0, cu_seqlens=None) -> SageShape:
-    s = SageShape(B, N, H, D, int(tok_stride), None, 0)
+def make_shape(B, N, H, D, tok_stride=0, cu_seqlens=None, q_gran="block64", k_gran="block64") -> SageShape:
+    """q_gran / k_gran: a GRAN name (or its integer code) for the Q / K scale groups."""
+    s = SageShape(B, N, H, D, int(tok_stride), None, 0, GRAN.get(q_gran, q_gran), GRAN.get(k_gran, k_gran))
     if cu_seqlens is not None:
         arr = (ctypes.c_int32 * len(cu_seqlens))(*[int(x) for x in cu_seqlens])
         s.cu_seqlens = ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32))
@@ -105,6 +110,12 @@ def _stream(stream) -> int | None:
 
 def npad(N: int) -> int:
     return int(_lib.sage_npad(int(N)))
+
+
+def scale_shape(B: int, H: int, N: int, gran="block64") -> tuple:
+    """Shape of a Q or K scale array: one per 64-token block, else one per token."""
+    Np = npad(N)
+    return (B, H, Np // 64) if GRAN.get(gran, gran) == GRAN["block64"] else (B, H, Np)
 
 
 def workspace_bytes(shape: SageShape) -> int:
@@ -159,16 +170,16 @@ class Buffers:
     """Device buffers of one shape for the whole path (torch allocates them)."""
 
     def __init__(self, B, N, H, D, device="cuda", out_fp32=False, with_lse=False, tok_stride=0,
-                 cu_seqlens=None):
-        self.shape = make_shape(B, N, H, D, tok_stride, cu_seqlens)
+                 cu_seqlens=None, q_gran="block64", k_gran="block64"):
+        self.shape = make_shape(B, N, H, D, tok_stride, cu_seqlens, q_gran, k_gran)
         self.B, self.N, self.H, self.D = B, N, H, D
         Np = npad(N)
         self.Npad = Np
         dev = torch.device(device)
         self.q_codes = torch.empty((B, H, Np, D), dtype=torch.int8, device=dev)
         self.k_codes = torch.empty((B, H, Np, D), dtype=torch.int8, device=dev)
-        self.q_scale = torch.empty((B, H, Np // 64), dtype=torch.float32, device=dev)
-        self.k_scale = torch.empty((B, H, Np // 64), dtype=torch.float32, device=dev)
+        self.q_scale = torch.empty(scale_shape(B, H, N, q_gran), dtype=torch.float32, device=dev)
+        self.k_scale = torch.empty(scale_shape(B, H, N, k_gran), dtype=torch.float32, device=dev)
         self.k_mean = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
         self.v_codes_t = torch.empty((B, H, D, Np), dtype=torch.uint8, device=dev)
         self.v_scale = torch.empty((B, H, D), dtype=torch.float32, device=dev)

@@ -8,12 +8,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 
 #include "sage.h"
 #include "sage_attn.cuh"
@@ -83,11 +85,17 @@ sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullpt
       e = cudaGetSymbolAddress(&p, g_sage_err);
       if (e == cudaSuccess) {
         ds.err_ptr = static_cast<int*>(p);
-        e = cudaFuncSetAttribute(sage::sage_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::AttnSmem<128>::kAlloc);
       }
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sage::sage_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::AttnSmem<64>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::AttnSmem<128>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::AttnSmem<64>::kAlloc);
       if (e == cudaSuccess && !g_encode) {
         void* fn = nullptr;
@@ -136,6 +144,12 @@ sage_status check_shape(const sage_shape& s, int64_t* tok_stride) {
   } else if (s.n_seg != 0) {
     return fail(SAGE_ERR_INVALID_ARG, "n_seg = %d without cu_seqlens", s.n_seg);
   }
+  for (const int g : {s.q_gran, s.k_gran})
+    if (g != SAGE_GRAN_BLOCK64 && g != SAGE_GRAN_TOKEN && g != SAGE_GRAN_SEGMENT64)
+      return fail(SAGE_ERR_INVALID_ARG, "q_gran / k_gran must be a sage_gran value (got %d)", g);
+  if ((s.q_gran == SAGE_GRAN_SEGMENT64 || s.k_gran == SAGE_GRAN_SEGMENT64) && s.n_seg > SAGE_MAX_SEGMENTS)
+    return fail(SAGE_ERR_UNSUPPORTED, "segment-local scale blocks take at most %d segments (got %d)",
+                SAGE_MAX_SEGMENTS, s.n_seg);
   *tok_stride = ts;
   return SAGE_OK;
 }
@@ -188,6 +202,81 @@ sage_status encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SAGE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return SAGE_OK;
+}
+
+static_assert(sage::kMaxSegments == SAGE_MAX_SEGMENTS, "segment table size");
+static_assert(sage::kGranBlock64 == SAGE_GRAN_BLOCK64 && sage::kGranToken == SAGE_GRAN_TOKEN &&
+                  sage::kGranSegment64 == SAGE_GRAN_SEGMENT64,
+              "granularity codes");
+
+// Segments of the shape (one segment [0, N) without cu_seqlens), then the
+// padding [N, Npad) as one more, with the number of 64-token blocks before each.
+void build_seg_table(const sage_shape& s, sage::SegTable* tab) {
+  std::memset(tab, 0, sizeof(*tab));
+  int n = 0, blocks = 0;
+  auto add = [&](int a, int e) {
+    tab->start[n] = a;
+    tab->gbase[n] = blocks;
+    blocks += (e - a + sage::kQKBlock - 1) / sage::kQKBlock;
+    ++n;
+    tab->start[n] = e;
+  };
+  if (s.cu_seqlens) {
+    for (int i = 0; i < s.n_seg; ++i) add(s.cu_seqlens[i], s.cu_seqlens[i + 1]);
+  } else {
+    add(0, s.N);
+  }
+  add(s.N, static_cast<int>(npad_of(s.N)));
+  tab->gbase[n] = blocks;
+  tab->n = n;
+}
+
+// The INT8 code pass of sage_quant_qk: the 64-token block kernel when both
+// tensors use blocks, the group kernel otherwise.
+void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const uint16_t* kb,
+                     const uint16_t* kmean, int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
+                     cudaStream_t cs) {
+  const int Npad = static_cast<int>(npad_of(s.N));
+  if (s.q_gran == SAGE_GRAN_BLOCK64 && s.k_gran == SAGE_GRAN_BLOCK64) {
+    const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
+    if (s.D == 128)
+      sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+                                                   k_codes, k_scale);
+    else
+      sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+                                                  k_codes, k_scale);
+    return;
+  }
+  sage::SegTable tab;
+  build_seg_table(s, &tab);
+  const int tiles = Npad / sage::kTile;
+  const int seg_ctas = (tab.gbase[tab.n] + 1) / 2;
+  int gx = 0;
+  for (const int g : {s.q_gran, s.k_gran}) gx = std::max(gx, g == SAGE_GRAN_SEGMENT64 ? seg_ctas : tiles);
+  const dim3 grid(gx, s.H, 2 * s.B);
+  // The nine (Q, K) granularity pairs, each for D = 64 and 128 (both block64:
+  // qk_block_quant above).
+  auto launch = [&](auto dq, auto dk) {
+    constexpr int GQ = decltype(dq)::value;
+    constexpr int GK = decltype(dk)::value;
+    if (s.D == 128)
+      sage::qk_group_quant<128, GQ, GK><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                                                              q_scale, k_codes, k_scale, tab);
+    else
+      sage::qk_group_quant<64, GQ, GK><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                                                             q_scale, k_codes, k_scale, tab);
+  };
+  using G0 = std::integral_constant<int, sage::kGranBlock64>;
+  using G1 = std::integral_constant<int, sage::kGranToken>;
+  using G2 = std::integral_constant<int, sage::kGranSegment64>;
+  auto with_k = [&](auto dq) {
+    if (s.k_gran == SAGE_GRAN_BLOCK64) launch(dq, G0{});
+    else if (s.k_gran == SAGE_GRAN_TOKEN) launch(dq, G1{});
+    else launch(dq, G2{});
+  };
+  if (s.q_gran == SAGE_GRAN_BLOCK64) with_k(G0{});
+  else if (s.q_gran == SAGE_GRAN_TOKEN) with_k(G1{});
+  else with_k(G2{});
 }
 
 template <int D>
@@ -273,7 +362,6 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
   uint16_t* kmean = reinterpret_cast<uint16_t*>(ws + lay.kmean);
   const int HD = s.H * s.D;
   const int nsb = (s.N + sage::kSumBlock - 1) / sage::kSumBlock;
-  const int Npad = static_cast<int>(npad_of(s.N));
   const uint16_t* qb = static_cast<const uint16_t*>(q);
   const uint16_t* kb = static_cast<const uint16_t*>(k);
 
@@ -281,11 +369,7 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
-  if (s.D == 128)
-    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
-  else
-    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  launch_qk_codes(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, cs);
   return launch_check("sage_quant_qk launch");
 }
 
@@ -376,14 +460,20 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   prm.nkv = static_cast<int>(Npad / sage::kBN);
   prm.sl2e = static_cast<float>(scale * 1.4426950408889634);
   prm.out_fp32 = out_fp32 ? 1 : 0;
+  prm.q_tok = s.q_gran != SAGE_GRAN_BLOCK64;
   prm.timeout_ns = g_timeout_ns.load();
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(static_cast<unsigned>(Npad / sage::kBM), s.H, s.B);
   (void)sm_count;
-  if (s.D == 128)
-    sage::sage_attn_kernel<128><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+  const bool k_tok = s.k_gran != SAGE_GRAN_BLOCK64;
+  if (s.D == 128 && !k_tok)
+    sage::sage_attn_kernel<128, false><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+  else if (s.D == 128)
+    sage::sage_attn_kernel<128, true><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+  else if (!k_tok)
+    sage::sage_attn_kernel<64, false><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
   else
-    sage::sage_attn_kernel<64><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+    sage::sage_attn_kernel<64, true><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
   return launch_check("sage_attn_fwd launch");
 }
 
@@ -451,7 +541,6 @@ sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int
   uint16_t* kmean = reinterpret_cast<uint16_t*>(scratch + psum_bytes);
   const int HD = s.H * s.D;
   const int nsb = static_cast<int>(nsb_sz);
-  const int Npad = static_cast<int>(npad_of(s.N));
   const uint16_t* qb = static_cast<const uint16_t*>(q);
   const uint16_t* kb = static_cast<const uint16_t*>(k);
   // Every scratch byte read below is written earlier in the same call.
@@ -459,11 +548,7 @@ sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
-  if (s.D == 128)
-    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
-  else
-    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes, k_scale);
+  launch_qk_codes(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, cs);
   return launch_check("sage_quant_qk_static launch");
 }
 

@@ -69,8 +69,8 @@ struct AttnSmem {
 };
 
 struct AttnParams {
-  const float* q_scale;   // [B*H, Npad/64]
-  const float* k_scale;   // [B*H, Npad/64]
+  const float* q_scale;   // [B*H, Npad/64] (64-token blocks) or [B*H, Npad] (q_tok)
+  const float* k_scale;   // [B*H, Npad/64], or [B*H, Npad] in the kKTok kernel
   const float* v_scale;   // [B*H, D]
   const float* v_mean;    // [B*H, D]
   void* out;              // [B, N, H, D] bf16 or f32
@@ -79,6 +79,7 @@ struct AttnParams {
   int N, H, Npad, nkv;
   float sl2e;             // sm_scale * log2(e)
   int out_fp32;
+  int q_tok;              // q_scale holds one scale per token
   int64_t timeout_ns;
 };
 
@@ -103,8 +104,9 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
 // accumulates y.  Every step is a binary32 operation with fixed rounding, so y
 // and its code equal the oracle's bit for bit.  kClamp: some u of this warp's
 // tile may be below -126.  pk[w] holds the codes of keys 4w .. 4w+3.
-template <bool kMasked, bool kClamp>
-__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], f32x2_t c2, f32x2_t e2, int valid,
+// cmul(p) gives the multipliers c of the quarter's keys 2p and 2p+1.
+template <bool kMasked, bool kClamp, class CMul>
+__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const CMul& cmul, f32x2_t e2, int valid,
                                                 const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
   // Stage-major over 8 pairs at a time: every step is issued for 8 independent
   // pairs before the next step, so consecutive instructions do not depend on
@@ -118,7 +120,7 @@ __device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], f32x2_t
       u[i] = x2_sub(x2_pack(s[2 * j], s[2 * j + 1]), k.round);   // exact integer S (the S bias is 1.5 * 2^23 too)
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) u[i] = x2_fma(u[i], c2, e2);
+    for (int i = 0; i < 8; ++i) u[i] = x2_fma(u[i], cmul(8 * h8 + i), e2);
     if (kClamp) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -178,12 +180,43 @@ __device__ __forceinline__ void chunk_minmax(const uint32_t (&a)[32], int valid,
              fmaxf(w[9], w[10]));
 }
 
+// One multiplier for every key of a quarter (its 64-key half shares one K scale).
+struct UniformMul {
+  f32x2_t c2;
+  __device__ __forceinline__ f32x2_t operator()(int) const { return c2; }
+};
+
+// Per-key multipliers c = RN(RN(qs * ks_j) * sl2e): lane L holds ks of key
+// 32 * quarter + L in kq, and a shuffle brings it to every row.
+struct KeyMul {
+  f32x2_t qs2, sl2e2;
+  float kq;
+  __device__ __forceinline__ f32x2_t operator()(int p) const {
+    const float k0 = __shfl_sync(0xFFFFFFFFu, kq, 2 * p);
+    const float k1 = __shfl_sync(0xFFFFFFFFu, kq, 2 * p + 1);
+    return x2_mul(x2_mul(x2_pack(__float_as_uint(k0), __float_as_uint(k1)), qs2), sl2e2);
+  }
+};
+
+struct HalfMuls {      // keys 0-63 use c0, keys 64-127 use c1
+  float c0, c1;
+  __device__ __forceinline__ UniformMul operator()(int qq) const { return UniformMul{x2_splat(qq < 2 ? c0 : c1)}; }
+};
+
+struct KeyMuls {       // per-key scales of the tile's four 32-key quarters
+  float qs, sl2e;
+  const float (&kq)[4];
+  __device__ __forceinline__ KeyMul operator()(int qq) const {
+    return KeyMul{x2_splat(qs), x2_splat(sl2e), kq[qq]};
+  }
+};
+
 // The exponential pass over a row's 128 scores in TMEM (taddr), 32 at a time;
 // each chunk's 32 codes go straight to
 // the row's 128B-swizzled P line (16-byte chunk q of row r lives at q ^ (r & 7)).
-// kSlow: masked keys or clamped exponents.
-template <bool kSlow>
-__device__ __forceinline__ void exp_pass(uint32_t taddr, float c0, float c1, float e, int valid,
+// kSlow: masked keys or clamped exponents.  muls(qq) gives quarter qq's multipliers.
+template <bool kSlow, class Muls>
+__device__ __forceinline__ void exp_pass(uint32_t taddr, const Muls& muls, float e, int valid,
                                          const Exp2Consts& ek, f32x2_t (&lsum)[4], uint8_t* prow, int row) {
   const f32x2_t e2 = x2_splat(e);
 #pragma unroll
@@ -192,15 +225,160 @@ __device__ __forceinline__ void exp_pass(uint32_t taddr, float c0, float c1, flo
     tmem_ld32(taddr + 32 * qq, cur);
     tmem_wait_ld();
     reg_fence(cur);
-    const f32x2_t c2 = x2_splat(qq < 2 ? c0 : c1);
     uint32_t pk[8];
-    softmax_quarter<kSlow, kSlow>(cur, c2, e2, valid - 32 * qq, ek, lsum, pk);
+    softmax_quarter<kSlow, kSlow>(cur, muls(qq), e2, valid - 32 * qq, ek, lsum, pk);
     *reinterpret_cast<uint4*>(prow + ((2 * qq) ^ (row & 7)) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     *reinterpret_cast<uint4*>(prow + ((2 * qq + 1) ^ (row & 7)) * 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
   }
 }
 
+// Tiles whose K scales differ inside a 64-key half (per-key multipliers; see
+// KeyMul); ks points at the tile's 128 per-key scales.
+//
+// Row max of t = RN(S_j * c_j) over the tile's valid keys.
+__device__ __forceinline__ float keywise_tile_max(uint32_t taddr, float qs, float sl2e, const float* ks, int valid) {
+  const int lane = threadIdx.x & 31;
+  float kq[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) kq[i] = ks[32 * i + lane];
+  float tmax = -__int_as_float(0x7F800000);
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    uint32_t cur[32];
+    tmem_ld32(taddr + 32 * qq, cur);
+    tmem_wait_ld();
+    reg_fence(cur);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float c = __fmul_rn(__fmul_rn(qs, __shfl_sync(0xFFFFFFFFu, kq[qq], i)), sl2e);
+      const float tv = __fmul_rn(__fsub_rn(__uint_as_float(cur[i]), kSBias), c);
+      if (32 * qq + i < valid) tmax = fmaxf(tmax, tv);
+    }
+  }
+  return tmax;
+}
+
+// The exponential pass of such a tile (always masked and clamped); returns the
+// tile's row sum of y = P~ * 448 as a pair (low + high is the sum).
+__device__ __forceinline__ f32x2_t keywise_exp_pass(uint32_t taddr, float qs, float sl2e, const float* ks, float e,
+                                                 int valid, uint8_t* prow, int row) {
+  const int lane = threadIdx.x & 31;
+  float kq[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) kq[i] = ks[32 * i + lane];
+  const Exp2Consts ek;
+  f32x2_t lsum[4] = {0, 0, 0, 0};
+  exp_pass<true>(taddr, KeyMuls{qs, sl2e, kq}, e, valid, ek, lsum, prow, row);
+  return x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
+}
+
+// One KV tile of a softmax thread's loop (thread = query row).  kKeywise: the
+// tile's K scales differ inside a 64-key half, so every key gets its own
+// multiplier (and the exponent is always clamped); the two instantiations are
+// separate code paths, so the rare per-key tiles leave the register allocation
+// of the common tiles alone.
 template <int D>
+struct SoftmaxTile {
+  uint64_t* bars;
+  volatile int* abort_flag;
+  int64_t tmo;
+  uint32_t ts, to;       // this warp's S and O columns in TMEM
+  float qs, sl2e;
+  const float* ks;       // per-key K scales of the head (per-key tiles only)
+  uint8_t* prow;         // this row of the shared P tile
+  int row;
+  float& m;              // running row max of t
+  float& l;              // running row sum of P~ * 448
+
+  // Returns false when a bounded wait gave up.
+  template <bool kKeywise>
+  __device__ __forceinline__ bool step(int j, int valid, float c0, float c1) {
+    const Exp2Consts ek;
+    if (!warp_wait(&bars[kBarSFull], static_cast<uint32_t>(j) & 1, abort_flag, tmo)) return false;
+    tc_fence_after();
+    // Row max of t = RN(S * c) (c > 0, so per block it is the max S scaled) and
+    // the per-block min S, which bounds every u from below.
+    float tmax, smin0 = 0.f, smin1 = 0.f;
+    if constexpr (kKeywise) {
+      tmax = keywise_tile_max(ts, qs, sl2e, ks + j * kBN, valid);
+    } else {
+      // Four 32-column loads, each issued while the previous chunk is reduced.
+      uint32_t ra[32], rb[32];
+      float mx[4], mn[4];
+      tmem_ld32(ts, ra);
+      tmem_wait_ld();
+      reg_fence(ra);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        uint32_t (&cur)[32] = (qq & 1) ? rb : ra;
+        uint32_t (&nxt)[32] = (qq & 1) ? ra : rb;
+        if (qq < 3) tmem_ld32(ts + 32 * (qq + 1), nxt);
+        if (valid >= kBN)
+          chunk_minmax<false>(cur, 32, mx[qq], mn[qq]);
+        else
+          chunk_minmax<true>(cur, valid - 32 * qq, mx[qq], mn[qq]);
+        if (qq < 3) {
+          tmem_wait_ld();
+          reg_fence(nxt);
+        }
+      }
+      tmax = __fmul_rn(__fsub_rn(fmaxf(mx[0], mx[1]), kSBias), c0);
+      if (valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(fmaxf(mx[2], mx[3]), kSBias), c1));
+      smin0 = __fsub_rn(fminf(mn[0], mn[1]), kSBias);
+      smin1 = __fsub_rn(fminf(mn[2], mn[3]), kSBias);
+    }
+    const float m_new = fmaxf(m, tmax);
+    const float alpha = exp2_fixed5(__fsub_rn(m, m_new));
+    const float e = __fsub_rn(kLog2P8, m_new);
+    // u is monotone in S (c > 0), so the smallest u of a block is its min S's;
+    // clamping is the identity unless that is below -126.
+    const bool clamp = kKeywise ||
+                       __any_sync(0xFFFFFFFFu, fminf(__fmaf_rn(smin0, c0, e), __fmaf_rn(smin1, c1, e)) < kExp2Min);
+    // P is single-buffered in shared memory: PV_{j-1} (issued right after QK_j)
+    // must have read it before this tile's codes are written.
+    if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) return false;
+    f32x2_t lsum[4] = {0, 0, 0, 0};
+    if constexpr (kKeywise)
+      lsum[0] = keywise_exp_pass(ts, qs, sl2e, ks + j * kBN, e, valid, prow, row);
+    else if (valid >= kBN && !clamp)
+      exp_pass<false>(ts, HalfMuls{c0, c1}, e, kBN, ek, lsum, prow, row);
+    else
+      exp_pass<true>(ts, HalfMuls{c0, c1}, e, valid, ek, lsum, prow, row);
+    // Re-seed S with the bias for the next tile's MMA, then release the buffer.
+    tmem_fill64(ts, kSBiasBits);
+    tmem_fill64(ts + 64, kSBiasBits);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&bars[kBarSEmpty]);
+    const f32x2_t ls2 = x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
+    l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(x2_lo(ls2), x2_hi(ls2)));
+
+    if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+      tc_fence_after();
+      const f32x2_t a2 = x2_splat(alpha);
+#pragma unroll
+      for (int cb = 0; cb < D; cb += 32) {
+        f32x2_t o[16];
+        tmem_ld32_pairs(to + cb, o);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] = x2_mul(o[i], a2);
+        tmem_st32_pairs(to + cb, o);
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(&bars[kBarPFull]);
+    m = m_new;
+    return true;
+  }
+};
+
+// kKTok: k_scale holds one scale per key (per-token or segment-local K
+// scales).  A tile whose K scales are equal within each 64-key half (the usual
+// case) runs exactly as with 64-token blocks; any other tile takes per-key
+// multipliers and always clamps.
+template <int D, bool kKTok>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
@@ -346,15 +524,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const uint32_t ts = tmem_s + lane_base;
     const uint32_t to = tmem_o + lane_base;
     const int nqb = prm.Npad / 64;
-    const float qs = prm.q_scale[static_cast<int64_t>(bh) * nqb + qt * 2 + (row >> 6)];
-    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * nqb;
+    const float qs = prm.q_tok ? prm.q_scale[static_cast<int64_t>(bh) * prm.Npad + qt * kBM + row]
+                               : prm.q_scale[static_cast<int64_t>(bh) * nqb + qt * 2 + (row >> 6)];
+    const float* ks = prm.k_scale + static_cast<int64_t>(bh) * (kKTok ? prm.Npad : nqb);
     const float sl2e = prm.sl2e;
     uint8_t* sP = smem + L::kP;
     const float kNegInf = -__int_as_float(0x7F800000);
     float m = kNegInf;
     float l = 0.f;                                // sum of P~ * 448
     bool ok = true;
-    const Exp2Consts ek;
     static_assert(kSBias == kExp2Round, "the S bias doubles as the exp2 rounding constant");
     // Seed S with the bias and release it for the first QK^T MMA.
     tmem_fill64(ts, kSBiasBits);
@@ -362,89 +540,37 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&bars[kBarSEmpty]);
+    SoftmaxTile<D> tile{bars, abort_flag, tmo, ts, to, qs, sl2e, ks, sP + row * 128, row, m, l};
     for (int j = 0; j < nkv; ++j) {
-      // Keys 0-63 and 64-127 of the tile are two scale blocks.
-      const float c0 = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
-      const float c1 = __fmul_rn(__fmul_rn(qs, ks[2 * j + 1]), sl2e);
-      if (!warp_wait(&bars[kBarSFull], static_cast<uint32_t>(j) & 1, abort_flag, tmo)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const int valid = min(kBN, prm.N - j * kBN);   // valid keys in this tile
-      // Row max of t = RN(S * c) (c > 0, so per block it is the max S scaled) and
-      // the per-block min S, which bounds every u from below.
-      float tmax, smin0, smin1;
-      {
-        // Four 32-column loads, each issued while the previous chunk is reduced.
-        uint32_t ra[32], rb[32];
-        float mx[4], mn[4];
-        tmem_ld32(ts, ra);
-        tmem_wait_ld();
-        reg_fence(ra);
+      float c0, c1;
+      bool keywise = false;      // kKTok: a 64-key half mixes K scales
+      if constexpr (kKTok) {
+        float kq[4];             // lane L: the scale of key 32 * i + L in kq[i]
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          uint32_t (&cur)[32] = (qq & 1) ? rb : ra;
-          uint32_t (&nxt)[32] = (qq & 1) ? ra : rb;
-          if (qq < 3) tmem_ld32(ts + 32 * (qq + 1), nxt);
-          if (valid >= kBN)
-            chunk_minmax<false>(cur, 32, mx[qq], mn[qq]);
-          else
-            chunk_minmax<true>(cur, valid - 32 * qq, mx[qq], mn[qq]);
-          if (qq < 3) {
-            tmem_wait_ld();
-            reg_fence(nxt);
-          }
-        }
-        tmax = __fmul_rn(__fsub_rn(fmaxf(mx[0], mx[1]), kSBias), c0);
-        if (valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(fmaxf(mx[2], mx[3]), kSBias), c1));
-        smin0 = __fsub_rn(fminf(mn[0], mn[1]), kSBias);
-        smin1 = __fsub_rn(fminf(mn[2], mn[3]), kSBias);
+        for (int i = 0; i < 4; ++i) kq[i] = ks[j * kBN + 32 * i + lane];
+        const float f0 = __shfl_sync(0xFFFFFFFFu, kq[0], 0);    // key 0 (always valid)
+        const float f1 = __shfl_sync(0xFFFFFFFFu, kq[2], 0);    // key 64
+        bool same = true;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) same = same && (32 * i + lane >= valid || kq[i] == (i < 2 ? f0 : f1));
+        keywise = !__all_sync(0xFFFFFFFFu, same);
+        c0 = __fmul_rn(__fmul_rn(qs, f0), sl2e);
+        c1 = __fmul_rn(__fmul_rn(qs, f1), sl2e);
+      } else {
+        // Keys 0-63 and 64-127 of the tile are two scale blocks.
+        c0 = __fmul_rn(__fmul_rn(qs, ks[2 * j]), sl2e);
+        c1 = __fmul_rn(__fmul_rn(qs, ks[2 * j + 1]), sl2e);
       }
-      const float m_new = fmaxf(m, tmax);
-      const float alpha = exp2_fixed5(__fsub_rn(m, m_new));
-      const float e = __fsub_rn(kLog2P8, m_new);
-      // u is monotone in S (c > 0), so the smallest u of a block is its min S's;
-      // clamping is the identity unless that is below -126.
-      const bool clamp = __any_sync(0xFFFFFFFFu, fminf(__fmaf_rn(smin0, c0, e), __fmaf_rn(smin1, c1, e)) < kExp2Min);
-      // P is single-buffered in shared memory: PV_{j-1} (issued right after QK_j)
-      // must have read it before this tile's codes are written.
-      if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) {
+      if (kKTok && keywise) {
+        if (!tile.template step<true>(j, valid, c0, c1)) {
+          ok = false;
+          break;
+        }
+      } else if (!tile.template step<false>(j, valid, c0, c1)) {
         ok = false;
         break;
       }
-      f32x2_t lsum[4] = {0, 0, 0, 0};
-      uint8_t* prow = sP + row * 128;
-      if (valid >= kBN && !clamp)
-        exp_pass<false>(ts, c0, c1, e, kBN, ek, lsum, prow, row);
-      else
-        exp_pass<true>(ts, c0, c1, e, valid, ek, lsum, prow, row);
-      // Re-seed S with the bias for the next tile's MMA, then release the buffer.
-      tmem_fill64(ts, kSBiasBits);
-      tmem_fill64(ts + 64, kSBiasBits);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars[kBarSEmpty]);
-      const f32x2_t ls2 = x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
-      l = __fadd_rn(__fmul_rn(l, alpha), __fadd_rn(x2_lo(ls2), x2_hi(ls2)));
-
-      if (j > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
-        tc_fence_after();
-        const f32x2_t a2 = x2_splat(alpha);
-#pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
-          f32x2_t o[16];
-          tmem_ld32_pairs(to + cb, o);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[i] = x2_mul(o[i], a2);
-          tmem_st32_pairs(to + cb, o);
-        }
-        tmem_wait_st();
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars[kBarPFull]);
-      m = m_new;
     }
     if (ok && warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(nkv - 1) & 1, abort_flag, tmo)) {
       tc_fence_after();

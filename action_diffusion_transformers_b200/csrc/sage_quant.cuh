@@ -322,6 +322,219 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
 }
 
 // ----------------------------------------------------------------------------
+// Q / K quantization at any scale granularity (64-token blocks, one scale per
+// token, 64-token blocks restarting at every segment start).  A CTA holds two
+// "slots" of up to 64 consecutive tokens of one (b, h): the two halves of a
+// 128-token tile for the block and token granularities, or two consecutive
+// segment-local blocks.  Thread mapping as in qk_block_quant.  The absmax is
+// reduced over the kLPR lanes of a token row (per token) or over the whole slot
+// (per block).  Block scales go to [B*H, Npad/64]; per-token and segment-local
+// scales to [B*H, Npad], every token holding its group's scale.
+// ----------------------------------------------------------------------------
+constexpr int kGranBlock64 = 0;
+constexpr int kGranToken = 1;
+constexpr int kGranSegment64 = 2;
+constexpr int kMaxSegments = 256;
+
+// The segments of a packed sequence, then the padding [N, Npad) as one more
+// segment; gbase[s] = number of 64-token blocks before segment s.  Passed by
+// value as a kernel parameter (2 KB).
+struct SegTable {
+  int n;                              // segments, the padding included
+  int start[kMaxSegments + 2];        // segment s is [start[s], start[s + 1])
+  int gbase[kMaxSegments + 2];        // gbase[n] = all blocks
+};
+
+// First token and length of segment-local block g (g < seg.gbase[seg.n]).
+__device__ __forceinline__ void seg_block(const SegTable& seg, int g, int& start, int& len) {
+  int lo = 0, hi = seg.n;               // largest s with gbase[s] <= g (empty segments skipped)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (seg.gbase[mid] <= g) lo = mid; else hi = mid;
+  }
+  start = seg.start[lo] + kQKBlock * (g - seg.gbase[lo]);
+  len = min(kQKBlock, seg.start[lo + 1] - start);
+}
+
+// One CTA of qk_group_quant: tensor K (is_k) or Q at granularity kGran.
+template <int D, int kGran>
+__device__ __forceinline__ void group_quant_cta(bool is_k, const uint16_t* __restrict__ q,
+                                                const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
+                                                int64_t tok_stride, const uint16_t* __restrict__ k_mean,
+                                                int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+                                                int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
+                                                const SegTable& seg) {
+  constexpr int gran = kGran;
+  constexpr int kLPR = D / 8;             // threads per token row
+  constexpr int kRPP = 256 / kLPR;        // token rows per pass
+  constexpr int kTPT = kTile / kRPP;      // token rows per thread (half in each slot)
+  constexpr int kHalf = kTPT / 2;
+  __shared__ float red[8][2];
+  const int h = is_k ? H - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
+  const int b = static_cast<int>(blockIdx.z) % B;
+  const uint16_t* src = is_k ? k : q;
+  const int cg = threadIdx.x % kLPR;
+  const int r0 = threadIdx.x / kLPR;
+  const int d0 = cg * 8;
+
+  int gstart[2], glen[2];
+  if constexpr (gran == kGranSegment64) {
+    const int G = seg.gbase[seg.n];
+    if (2 * static_cast<int>(blockIdx.x) >= G) return;   // the whole CTA leaves
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int g = 2 * blockIdx.x + s;
+      gstart[s] = 0;
+      glen[s] = 0;
+      if (g < G) seg_block(seg, g, gstart[s], glen[s]);
+    }
+  } else {
+    if (static_cast<int>(blockIdx.x) >= Npad / kTile) return;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      gstart[s] = blockIdx.x * kTile + s * kQKBlock;
+      glen[s] = kQKBlock;
+    }
+  }
+
+  float mean[8];
+  if (is_k) {
+    const uint4 mraw = *reinterpret_cast<const uint4*>(k_mean + (static_cast<int64_t>(b) * H + h) * D + d0);
+    unpack8(mraw, mean);
+  }
+  uint4 raw[kTPT];
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int o = r0 + (t % kHalf) * kRPP;
+    const int n = gstart[t / kHalf] + o;
+    raw[t] = (o < glen[t / kHalf] && n < N)
+                 ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
+                 : make_uint4(0u, 0u, 0u, 0u);
+  }
+  float x[kTPT][8];
+  float rmax[kTPT];
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int o = r0 + (t % kHalf) * kRPP;
+    const int n = gstart[t / kHalf] + o;
+    unpack8(raw[t], x[t]);
+    if (is_k && o < glen[t / kHalf] && n < N) {
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) {
+        const __nv_bfloat162 c2 =
+            __floats2bfloat162_rn(__fsub_rn(x[t][i], mean[i]), __fsub_rn(x[t][i + 1], mean[i + 1]));
+        x[t][i] = __low2float(c2);
+        x[t][i + 1] = __high2float(c2);
+      }
+    }
+    rmax[t] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rmax[t] = fmaxf(rmax[t], fabsf(x[t][i]));
+  }
+  const int64_t bh = static_cast<int64_t>(b) * H + h;
+  int8_t* dst = is_k ? k_codes : q_codes;
+  float* sdst = is_k ? k_scale : q_scale;
+  float inv[kTPT];
+  if constexpr (gran == kGranToken) {
+    // The kLPR lanes of one token row are consecutive lanes of one warp; after
+    // the butterfly every one of them holds the absmax of all kTPT rows.  Lane
+    // cg < kTPT then forms the scale of row cg (and stores it), lane kTPT + t
+    // the inverse of row t: one division per lane, the inverses shuffled out.
+    static_assert(2 * kTPT == kLPR, "one division per lane");
+#pragma unroll
+    for (int t = 0; t < kTPT; ++t) {
+#pragma unroll
+      for (int o = kLPR / 2; o >= 1; o >>= 1) rmax[t] = fmaxf(rmax[t], __shfl_xor_sync(0xFFFFFFFFu, rmax[t], o));
+    }
+    const int mine = cg % kTPT;
+    float a = rmax[0];
+#pragma unroll
+    for (int t = 1; t < kTPT; ++t) a = mine == t ? rmax[t] : a;
+    const bool is_scale = cg < kTPT;
+    const float val = a > 0.f ? __fdiv_rn(is_scale ? a : 127.f, is_scale ? 127.f : a) : 0.f;
+    const int base = (threadIdx.x & 31) & ~(kLPR - 1);
+#pragma unroll
+    for (int t = 0; t < kTPT; ++t) inv[t] = __shfl_sync(0xFFFFFFFFu, val, base + kTPT + t);
+    if (is_scale) {
+      const int o = r0 + (mine % kHalf) * kRPP;
+      const int s = mine / kHalf;
+      const int gs = s == 0 ? gstart[0] : gstart[1];
+      const int gl = s == 0 ? glen[0] : glen[1];
+      if (o < gl) sdst[bh * Npad + gs + o] = val;
+    }
+  } else {
+    float amax[2] = {0.f, 0.f};
+#pragma unroll
+    for (int t = 0; t < kTPT; ++t) amax[t / kHalf] = fmaxf(amax[t / kHalf], rmax[t]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      amax[0] = fmaxf(amax[0], __shfl_xor_sync(0xFFFFFFFFu, amax[0], o));
+      amax[1] = fmaxf(amax[1], __shfl_xor_sync(0xFFFFFFFFu, amax[1], o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      red[threadIdx.x >> 5][0] = amax[0];
+      red[threadIdx.x >> 5][1] = amax[1];
+    }
+    __syncthreads();
+    float scale[2], sinv[2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      float a = red[0][s];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][s]);
+      scale[s] = 0.f;
+      sinv[s] = 0.f;
+      if (a > 0.f) {
+        scale[s] = __fdiv_rn(a, 127.f);
+        sinv[s] = __fdiv_rn(127.f, a);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kTPT; ++t) inv[t] = sinv[t / kHalf];
+    if constexpr (gran == kGranBlock64) {
+      if (threadIdx.x < 2)
+        sdst[bh * (Npad / kQKBlock) + blockIdx.x * 2 + threadIdx.x] = threadIdx.x == 0 ? scale[0] : scale[1];
+    } else if (cg == 0) {
+#pragma unroll
+      for (int t = 0; t < kTPT; ++t) {
+        const int o = r0 + (t % kHalf) * kRPP;
+        if (o < glen[t / kHalf]) sdst[bh * Npad + gstart[t / kHalf] + o] = scale[t / kHalf];
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int o = r0 + (t % kHalf) * kRPP;
+    if (o >= glen[t / kHalf]) continue;
+    const int n = gstart[t / kHalf] + o;
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int c = rne_small(__fmul_rn(x[t][i], inv[t]));
+      c = max(-127, min(127, c));
+      w[i >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w[0], w[1]);
+  }
+}
+
+// Grid (max CTAs of the two tensors, H, 2B): z < B quantizes K at kGranK, the
+// rest Q at kGranQ.  A CTA past its tensor's tiles or blocks leaves at once.
+template <int D, int kGranQ, int kGranK>
+__global__ void __launch_bounds__(256, (kGranQ == kGranSegment64 || kGranK == kGranSegment64) ? 2 : 3)
+    qk_group_quant(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
+                   int64_t tok_stride, const uint16_t* __restrict__ k_mean, int8_t* __restrict__ q_codes,
+                   float* __restrict__ q_scale, int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
+                   const __grid_constant__ SegTable seg) {
+  if (static_cast<int>(blockIdx.z) < B)
+    group_quant_cta<D, kGranK>(true, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes, k_scale,
+                               seg);
+  else
+    group_quant_cta<D, kGranQ>(false, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes,
+                               k_scale, seg);
+}
+
+// ----------------------------------------------------------------------------
 // V centre + E4M3 quantization + transpose.  CTA = one (b, h, 128-token tile).
 // Phase 1: threads read 16-byte pieces of token rows, quantize 8 channels and
 // store the 8 code bytes into a [128][D] shared tile.  Phase 2: each thread

@@ -7,6 +7,7 @@ BF16 NHD; synthetic, seeded).  Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload action_dit|mid_video|long_video|ragged|tiny]
+                    [--q-gran block64|token|segment64] [--k-gran block64|token|segment64]
 
 value      = attention ops (4*B*H*N^2*D, INT8 QK^T + FP8 PV) per step, all ranks,
              / device time of the whole step (quant + attention), in TOPS;
@@ -60,7 +61,7 @@ def attn_traffic(workload: str):
     pkg = os.path.join(ROOT, "action_diffusion_transformers_b200")
     try:
         with open(os.path.join(pkg, "ncu_counters.json")) as f:
-            rec = json.load(f)["sage_attn_kernel<128>"]
+            rec = json.load(f)["sage_attn_kernel<128, false>"]
     except (OSError, KeyError, ValueError):
         return None
     h = hashlib.sha256()
@@ -80,17 +81,23 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="action_dit", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--q-gran", default="block64", choices=["block64", "token", "segment64"],
+                    help="INT8 scale groups of Q (default: 64-token blocks)")
+    ap.add_argument("--k-gran", default="block64", choices=["block64", "token", "segment64"],
+                    help="INT8 scale groups of K (default: 64-token blocks)")
     ap.add_argument("--peaks", action="store_true",
                     help="measure library INT8 / FP8 / BF16 GEMM throughput at 8192^3 and exit")
     return ap.parse_args()
 
 
-def quant_bytes(w):
-    """Algorithmic bytes of the two quantization calls (per step)."""
+def quant_bytes(w, q_gran="block64", k_gran="block64"):
+    """Algorithmic bytes of the two quantization calls (per step): 4 B per Q/K
+    scale, one per 64-token block or one per (padded) token."""
     elems = w.B * w.N * w.H * w.D
-    blocks = w.B * w.H * ((w.N + 127) // 128 * 2)
+    npad = (w.N + 127) // 128 * 128
+    scales = sum(w.B * w.H * (npad // 64 if g == "block64" else npad) for g in (q_gran, k_gran))
     chans = w.B * w.H * w.D
-    qk = elems * (2 + 2 + 1 + 1) + blocks * 4 * 2 + chans * 2
+    qk = elems * (2 + 2 + 1 + 1) + scales * 4 + chans * 2
     v = elems * (2 + 1) + chans * 8
     return qk, v
 
@@ -173,13 +180,13 @@ def gpu_id_for(dev_index: int):
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_sample(w, qb, kb, vb, rows: int, heads: int):
+def oracle_sample(w, qb, kb, vb, rows: int, heads: int, q_gran="block64", k_gran="block64"):
     """Time the CPU oracle on `heads` heads of batch 0 (full quantization of those
     heads, attention for `rows` query rows).  Returns (ops, seconds)."""
     from oracle import sage_oracle as so
     t0 = time.perf_counter()
     sl = (slice(0, 1), slice(None), slice(0, heads), slice(None))
-    qk = so.quant_qk(qb[sl], kb[sl])
+    qk = so.quant_qk(qb[sl], kb[sl], q_gran, k_gran, w.cu_seqlens)
     vv = so.quant_v(vb[sl])
     r = synth.sample_rows(w.N, rows, 0)[:rows] if rows < w.N else None
     so.attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"], vv["v_codes_t"], vv["v_scale"],
@@ -204,12 +211,13 @@ def run_reference(args, rank):
     w = synth.WORKLOADS[args.workload]
     qb, kb, vb = synth.generate(w)
     rows, heads = 256, 1
+    grans = (args.q_gran, args.k_gran)
     for _ in range(args.warmup):
-        oracle_sample(w, qb, kb, vb, rows, heads)
+        oracle_sample(w, qb, kb, vb, rows, heads, *grans)
     times = []
     ops = 0.0
     for _ in range(args.steps):
-        ops, dt = oracle_sample(w, qb, kb, vb, rows, heads)
+        ops, dt = oracle_sample(w, qb, kb, vb, rows, heads, *grans)
         times.append(dt)
     tot = sum(times)
     value = ops * len(times) / tot / 1e12
@@ -218,7 +226,8 @@ def run_reference(args, rank):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32/f64 (CPU oracle)", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D},
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D,
+                       "q_gran": args.q_gran, "k_gran": args.k_gran},
             "cpu_baseline": {"value": value, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -287,7 +296,7 @@ def main():
     qb, kb, vb = synth.generate(w)
     as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
     q, k, v = as_dev(qb), as_dev(kb), as_dev(vb)
-    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens)
+    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=args.q_gran, k_gran=args.k_gran)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
@@ -369,15 +378,16 @@ def main():
     # --------------------------------------------------------------- roofline, baseline
     peaks, src = load_peaks()
     peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    k_blocks = args.k_gran == "block64"
     attn_mean_ms = statistics.mean(at_ms)
     achieved = ops / (attn_mean_ms / 1e3) / 1e12
-    qk_bytes, v_bytes = quant_bytes(w)
+    qk_bytes, v_bytes = quant_bytes(w, args.q_gran, args.k_gran)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of CPU work on the GPU machine's host: 4 heads, 2^26 (query row, key) pairs
         heads = min(4, w.H)
         rows = max(1, min(w.N, (1 << 26) // (heads * w.N)))
-        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads)
+        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads, args.q_gran, args.k_gran)
         cpu = {"value": o_ops / o_dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{heads} heads of batch 0: full K/V quantization of those heads + attention for "
                          f"{rows} query rows each ({o_dt:.1f} s)"}
@@ -391,9 +401,11 @@ def main():
         "warmup": args.warmup, "ms_per_step": max_total_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "global_batch": w.B * world,
-                   "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)"},
+                   "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)",
+                   "q_gran": args.q_gran, "k_gran": args.k_gran},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": attn_traffic(w.name), "kernel": "sage_attn_kernel<128>",
+                     "frac": achieved / peak, "traffic": attn_traffic(w.name) if k_blocks else None,
+                     "kernel": f"sage_attn_kernel<{w.D}, {'false' if k_blocks else 'true'}>",
                      "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"},
         "kernels_us": {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
                        "attn": 1e3 * attn_mean_ms},

@@ -65,17 +65,45 @@ typedef enum {
   SAGE_ERR_WORKSPACE = 6       /* workspace missing or smaller than needed   */
 } sage_status;
 
+/* INT8 scale granularity of Q or K (the groups of tokens that share one
+ * scale; every group spans all D channels of one (b, h)).
+ *  SAGE_GRAN_BLOCK64    64-token blocks on one grid over the whole sequence
+ *                       (the configurations' "Q/K INT8 blocks 64 tokens").
+ *                       Scales: f32 [B, H, Npad/64], one per block.
+ *  SAGE_GRAN_TOKEN      one scale per token.  On these tensor cores one thread
+ *                       owns one query row, so this is the counterpart of the
+ *                       per-thread granularity named in "FLUX.3 Action RTX
+ *                       5090 report", card 03.  Scales: f32 [B, H, Npad].
+ *  SAGE_GRAN_SEGMENT64  64-token blocks restarting at every segment start of
+ *                       cu_seqlens (a block never mixes two streams of a
+ *                       packed joint sequence; a segment's last block may be
+ *                       short); the padding [N, Npad) continues the 64-token
+ *                       grid from N.  Scales: f32 [B, H, Npad], every token
+ *                       holding its block's scale.  At most SAGE_MAX_SEGMENTS
+ *                       segments; without cu_seqlens the one segment is [0, N).
+ * Padded tokens always get scale 0 and zero codes.  sage_quant_qk writes and
+ * sage_attn_fwd reads the layouts that the shape's q_gran / k_gran select, so
+ * both calls must be given the same values. */
+typedef enum {
+  SAGE_GRAN_BLOCK64 = 0,
+  SAGE_GRAN_TOKEN = 1,
+  SAGE_GRAN_SEGMENT64 = 2
+} sage_gran;
+#define SAGE_MAX_SEGMENTS 256
+
 typedef struct {
   int B, N, H, D;
   int64_t tok_stride;         /* elements between consecutive tokens of the
                                  call's BF16 input(s); 0 means H*D           */
   const int32_t* cu_seqlens;  /* HOST pointer to n_seg+1 segment offsets of a
                                  packed joint sequence, or NULL.  Validated
-                                 (starts at 0, non-decreasing, ends at N) and
-                                 otherwise informational: attention is full
-                                 over the concatenation and the K/V means run
-                                 over all N tokens.                          */
+                                 (starts at 0, non-decreasing, ends at N).
+                                 Attention is full over the concatenation and
+                                 the K/V means run over all N tokens; the
+                                 offsets only place SAGE_GRAN_SEGMENT64 blocks. */
   int n_seg;
+  int q_gran;                 /* sage_gran of the Q scales (0: 64-token blocks) */
+  int k_gran;                 /* sage_gran of the K scales (0: 64-token blocks) */
 } sage_shape;
 
 /* N rounded up to a whole 128-row tile. */
@@ -91,14 +119,15 @@ SAGE_API size_t sage_workspace_bytes(sage_shape s);
  *
  * in : q, k        BF16 [B, N, H, D] with s.tok_stride (both tensors).
  * out: q_codes     int8 [B, H, Npad, D]; rows >= N are 0.
- *      q_scale     f32  [B, H, Npad/64]; blocks past N are 0.
- *      k_codes     int8 [B, H, Npad, D]; k_scale f32 [B, H, Npad/64].
+ *      q_scale     f32  [B, H, Npad/64] (s.q_gran 64-token blocks) or
+ *                  [B, H, Npad] (per token, segment-local blocks); 0 past N.
+ *      k_codes     int8 [B, H, Npad, D]; k_scale f32 as q_scale, by s.k_gran.
  *      k_mean      BF16 [B, H, D] or NULL.
  * Rule: mean_k[b,h,d] = RN_bf16(sum_n k / N), the FP64 sum taken in a fixed
  * order (64-token blocks in token order; 32 interleaved lanes over blocks;
  * butterfly 16,8,4,2,1 over lanes) and the quotient rounded once to BF16;
- * kc = RN_bf16(RN_f32(k - mean_k)).  For each 64-token block of one (b,h)
- * over all D: amax = max|x|, scale = RN(amax/127), inv = RN(127/amax),
+ * kc = RN_bf16(RN_f32(k - mean_k)).  For each scale group (sage_gran) of one
+ * (b,h) over all D: amax = max|x|, scale = RN(amax/127), inv = RN(127/amax),
  * code = clamp(RNE(RN(x*inv)), -127, 127); amax == 0 gives 0 scale and codes.
  * Q is quantized as is, K after centring.  Codes are bit-exact with that rule.
  * workspace: >= sage_workspace_bytes(s) bytes of device memory, 256-B aligned.
@@ -131,12 +160,15 @@ SAGE_API sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_
  * accumulation, V mean added back; "MiniMax H3 on DGX Spark", 01.)
  *
  * in : the outputs of sage_quant_qk / sage_quant_v for the same shape
- *      (s.tok_stride is ignored here).
+ *      (s.tok_stride is ignored here; s.q_gran and s.k_gran give the layouts
+ *      of q_scale and k_scale).
  *      sm_scale <= 0 selects 1/sqrt(D).
  * out: out   [B, N, H, D], BF16 (out_fp32 == 0) or FP32 (out_fp32 != 0).
  *      lse   f32 [B, H, N] natural-log softmax denominator, or NULL.
  * Per 128-row query tile and 128-key tile: S = Qc Kc^T exactly in INT32 on the
- * tensor cores; t = S * qs * ks * sm_scale * log2(e) in FP32; running row max m;
+ * tensor cores; t = S * c in FP32 with c = RN(RN(qs_i * ks_j) * RN(sm_scale *
+ * log2 e)), qs_i / ks_j the scales of the groups holding query i / key j;
+ * running row max m;
  * P~ = exp2(t - m) in [0, 1]; l accumulates unquantized P~; P8 = E4M3(P~*448);
  * O_acc = O_acc * exp2(m_old - m_new) + P8 V8 (FP8 MMA, FP32 accumulation);
  * O = O_acc * (v_scale/448) / l + v_mean.  Keys >= N are masked.  Matches the

@@ -76,8 +76,30 @@ def test_cu_seqlens_validation(adt):
     for s in (bad_end, bad_order, bad_start):
         assert _qk(adt, s) == 1
     # valid arguments get past validation; without a GPU the device lookup fails
-    st = _qk(adt, ok)
-    assert st in (0, 4)
+    # (with a GPU the fake pointers would reach a kernel, so that leg is skipped)
+    if not _gpu_present():
+        assert _qk(adt, ok) == 4
+
+
+def _gpu_present():
+    import torch
+    return torch.cuda.is_available()
+
+
+def test_granularity_validation(adt):
+    for q_gran, k_gran in ((3, 0), (0, -1), (7, 7)):
+        assert _qk(adt, adt.make_shape(1, 256, 2, 64, q_gran=q_gran, k_gran=k_gran)) == 1
+        assert b"gran" in adt._lib.sage_last_error()
+    many = list(range(0, 258)) + [300]                 # 258 segments
+    assert _qk(adt, adt.make_shape(1, 300, 2, 64, cu_seqlens=many, k_gran="segment64")) == 2
+    assert b"segments" in adt._lib.sage_last_error()
+    assert _qk(adt, adt.make_shape(1, 300, 2, 64, cu_seqlens=many, q_gran="segment64")) == 2
+    limit = list(range(0, 256)) + [300]                # 256 segments: accepted
+    if not _gpu_present():
+        assert _qk(adt, adt.make_shape(1, 300, 2, 64, cu_seqlens=limit, k_gran="segment64")) == 4
+        assert _qk(adt, adt.make_shape(1, 300, 2, 64, cu_seqlens=many)) == 4   # blocks ignore the count
+    assert adt.scale_shape(2, 3, 200, "block64") == (2, 3, 4)
+    assert adt.scale_shape(2, 3, 200, "token") == adt.scale_shape(2, 3, 200, "segment64") == (2, 3, 256)
 
 
 def test_attn_and_v_validation(adt):

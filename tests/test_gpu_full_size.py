@@ -12,7 +12,9 @@ the oracle computes head by head and row by row:
   per-token INT8 variant) reaches about 0.998, so the check is >= 0.997;
 * the BF16 output equals the RNE rounding of the FP32 output on those rows;
 * the LSE of those rows within 1e-4 (relative to max(1, |lse|)) of the oracle's.
-A D = 64 shape with many KV tiles and a ragged tail runs the same checks.
+A D = 64 shape with many KV tiles and a ragged tail runs the same checks, and
+so does the ragged joint sequence with segment-local K blocks and per-token
+or segment-local Q scales.
 """
 import numpy as np
 import pytest
@@ -44,15 +46,19 @@ def _cos(a, b):
     return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
 
 
-@pytest.mark.parametrize("name", ["action_dit", "mid_video", "long_video", "ragged", "d64_many_tiles"])
-def test_full_size_sampled_parity(adt, name):
+@pytest.mark.parametrize("name,q_gran,k_gran", [
+    ("action_dit", "block64", "block64"), ("mid_video", "block64", "block64"),
+    ("long_video", "block64", "block64"), ("ragged", "block64", "block64"),
+    ("d64_many_tiles", "block64", "block64"),
+    ("ragged", "token", "segment64"), ("ragged", "segment64", "segment64")])
+def test_full_size_sampled_parity(adt, name, q_gran, k_gran):
     if name == "d64_many_tiles":
         w = synth.custom(1, 8200, 8, 64, seed=7, k_sigma=4.0, v_sigma=1.0, outlier_frac=0.02)
     else:
         w = synth.WORKLOADS[name]
     qb, kb, vb = synth.generate(w)
     q, k, v = _dev(qb), _dev(kb), _dev(vb)
-    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens)
+    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=q_gran, k_gran=k_gran)
     out16 = buf.run(q, k, v)
     out32 = torch.empty((w.B, w.N, w.H, w.D), dtype=torch.float32, device="cuda")
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
@@ -64,7 +70,7 @@ def test_full_size_sampled_parity(adt, name):
     rows = _rows(w.N, w.seed)
     for i, (b, h) in enumerate(heads):
         sl = (slice(b, b + 1), slice(None), slice(h, h + 1), slice(None))
-        ref_qk = so.quant_qk(qb[sl], kb[sl])
+        ref_qk = so.quant_qk(qb[sl], kb[sl], q_gran, k_gran, w.cu_seqlens)
         ref_v = so.quant_v(vb[sl])
         got = lambda t: t[b:b + 1, h:h + 1].cpu().numpy()  # noqa: E731
         assert np.array_equal(got(buf.q_codes), ref_qk["q_codes"])
