@@ -205,10 +205,13 @@ def k_mean_bf16(k_bits: np.ndarray) -> np.ndarray:
 
 
 def quant_qk(q_bits: np.ndarray, k_bits: np.ndarray, q_gran: str = "block64",
-             k_gran: str = "block64", cu_seqlens=None):
+             k_gran: str = "block64", cu_seqlens=None, normrope=None):
     """A1-A3: K smoothing and INT8 quantization of Q and K.
 
     q_bits, k_bits: BF16 bit patterns uint16 [B, N, H, D].
+    normrope: None, or dict(q_w, k_w, eps, cos, sin): Q and K are first taken
+    through RMSNorm and RoPE in BF16 (oracle.normrope.norm_rope_bf16), and
+    everything below runs on the result.
     K is centred by its BF16 token mean (over all N tokens, whatever the scale
     granularity) and rounded back to BF16 before quantization:
     kc = RN_bf16(RN32(k - mean_k)).  Q is quantized raw (the pages keep only K
@@ -217,6 +220,11 @@ def quant_qk(q_bits: np.ndarray, k_bits: np.ndarray, q_gran: str = "block64",
     quant_scales) and k_mean (uint16 [B, H, D]).
     """
     N = q_bits.shape[1]
+    if normrope is not None:
+        from .normrope import norm_rope_bf16
+        nr = normrope
+        q_bits = norm_rope_bf16(q_bits, nr["q_w"], nr["eps"], nr["cos"], nr["sin"])
+        k_bits = norm_rope_bf16(k_bits, nr["k_w"], nr["eps"], nr["cos"], nr["sin"])
     q32 = bf16_bits_to_f32(q_bits)
     k32 = bf16_bits_to_f32(k_bits)
     mean_bits = k_mean_bf16(k_bits)

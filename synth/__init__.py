@@ -29,6 +29,13 @@ Recipe (one numpy PCG64 generator per call, draws in this order):
     indices whose every value is replaced by a Student-t(3) draw (before the
     K offset is added, so the offset stays a per-channel shift);
  6. round to BF16 (RNE) and keep the raw uint16 bit patterns.
+
+Inputs of the fused QK RMSNorm + RoPE step (projection_outputs,
+normrope_inputs): Q and K before the norm (each token vector scaled by a
+log-normal factor), RMSNorm weights near 1, and the cos / sin tables of the
+tokens' (t, h, w, l) positions.  The tables are built here, in float64 rounded
+once to float32, because they are an input of that step (a model computes them
+once per sequence layout); the step itself (norm, rotation, rounding) is not.
 """
 from __future__ import annotations
 
@@ -136,3 +143,78 @@ def sample_rows(N: int, count: int, seed: int) -> np.ndarray:
         if pool.size:
             fixed = sorted(set(fixed) | set(rng.choice(pool, size=min(extra, pool.size), replace=False).tolist()))
     return np.asarray(fixed, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------- norm / RoPE inputs
+ROPE_THETA = 10000.0
+
+
+def rope_axes(D: int) -> tuple:
+    """Channel pairs given to each of the four RoPE axes (t, h, w, l): D/8 each.
+    The pages name the four axes but not their widths; equal widths are the
+    plainest reading."""
+    return (D // 8,) * 4
+
+
+def rope_positions(N: int, cu_seqlens=None, grid_w: int = 32, grid_h: int = 32) -> np.ndarray:
+    """Integer (t, h, w, l) positions [N, 4] of a packed joint sequence.
+
+    Without cu_seqlens the sequence is one video latent in raster order (w
+    fastest, then h, then t).  With cu_seqlens the first segment is text
+    (position l = index in the segment, t = h = w = 0) and every other segment
+    is a video latent of its own, in raster order from (0, 0, 0)."""
+    pos = np.zeros((N, 4), dtype=np.int64)
+    segs = [(0, N)] if cu_seqlens is None else list(zip(cu_seqlens[:-1], cu_seqlens[1:]))
+    for s, (a, e) in enumerate(segs):
+        i = np.arange(e - a)
+        if cu_seqlens is not None and s == 0:
+            pos[a:e, 3] = i
+        else:
+            pos[a:e, 0] = i // (grid_w * grid_h)
+            pos[a:e, 1] = (i // grid_w) % grid_h
+            pos[a:e, 2] = i % grid_w
+    return pos
+
+
+def rope_tables(pos: np.ndarray, D: int, theta: float = ROPE_THETA):
+    """cos, sin tables (float32 [N, D/2]) of the 4-axis rotary embedding.
+
+    Axis k owns the next rope_axes(D)[k] channel pairs; its pair j turns by
+    pos[:, k] * theta ** (-j / pairs_k), formed in float64 and rounded once
+    to float32 (cos and sin alike)."""
+    cols = []
+    for k, pairs in enumerate(rope_axes(D)):
+        freq = theta ** (-np.arange(pairs, dtype=np.float64) / pairs)
+        cols.append(pos[:, k:k + 1].astype(np.float64) * freq[None, :])
+    ang = np.concatenate(cols, axis=1)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def norm_weights(D: int, seed: int):
+    """RMSNorm weights of Q and K: BF16 bit patterns [D], near 1 (random init)."""
+    rng = np.random.default_rng(50_000 + seed)
+    wq = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    wk = (1.0 + 0.1 * rng.standard_normal(D)).astype(np.float32)
+    return to_bf16_bits(wq), to_bf16_bits(wk)
+
+
+def normrope_inputs(w: Workload, eps: float = 1e-6) -> dict:
+    """The inputs of the fused QK norm + RoPE step for a workload: weights,
+    eps (binary32) and the cos / sin tables of its token positions."""
+    q_w, k_w = norm_weights(w.D, w.seed)
+    cos, sin = rope_tables(rope_positions(w.N, w.cu_seqlens), w.D)
+    return dict(q_w=q_w, k_w=k_w, eps=float(np.float32(eps)), cos=cos, sin=sin)
+
+
+def projection_outputs(w: Workload):
+    """Q and K as they leave the projection (before the norm): the workload's
+    Q / K with a per-token magnitude spread (log-normal, sigma 1), the scale
+    that RMSNorm removes.  BF16 bit patterns [B, N, H, D]."""
+    q, k, _ = generate(w)
+    rng = np.random.default_rng(60_000 + w.seed)
+    out = []
+    for x in (q, k):
+        f = bits_to_f64(x).astype(np.float32)
+        f *= np.exp(rng.standard_normal((w.B, w.N, w.H, 1))).astype(np.float32)
+        out.append(to_bf16_bits(f))
+    return out[0], out[1]
