@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
                 4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_DEVICE_TIMEOUT", 6: "SAGE_ERR_WORKSPACE"}
 EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
             "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error",
-            "sage_quant_qk_static")
+            "sage_quant_qk_static", "sage_quant_qk_normrope")
 QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -45,6 +45,11 @@ class SageShape(ctypes.Structure):
                 ("n_seg", ctypes.c_int), ("q_gran", ctypes.c_int), ("k_gran", ctypes.c_int)]
 
 
+class SageNormRope(ctypes.Structure):
+    _fields_ = [("q_weight", ctypes.c_void_p), ("k_weight", ctypes.c_void_p), ("rope_cos", ctypes.c_void_p),
+                ("rope_sin", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 _vp = ctypes.c_void_p
 _lib.sage_npad.argtypes = [ctypes.c_int]
 _lib.sage_npad.restype = ctypes.c_size_t
@@ -54,6 +59,9 @@ _lib.sage_quant_qk.argtypes = [_vp, _vp, SageShape, _vp, _vp, _vp, _vp, _vp, _vp
 _lib.sage_quant_qk.restype = ctypes.c_int
 _lib.sage_quant_qk_static.argtypes = [_vp, _vp, SageShape, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.sage_quant_qk_static.restype = ctypes.c_int
+_lib.sage_quant_qk_normrope.argtypes = [_vp, _vp, SageShape, ctypes.POINTER(SageNormRope), _vp, _vp, _vp, _vp, _vp,
+                                        _vp, ctypes.c_size_t, _vp]
+_lib.sage_quant_qk_normrope.restype = ctypes.c_int
 _lib.sage_quant_v.argtypes = [_vp, SageShape, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_v.restype = ctypes.c_int
 _lib.sage_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, SageShape, ctypes.c_float, _vp, ctypes.c_int,
@@ -137,6 +145,18 @@ def sage_quant_qk_static(q, k, shape, q_codes, q_scale, k_codes, k_scale, k_mean
                                   _ptr(k_scale), _ptr(k_mean), _stream(stream)), "sage_quant_qk_static")
 
 
+def sage_quant_qk_normrope(q, k, shape, q_weight, k_weight, rope_cos, rope_sin, eps, q_codes, q_scale, k_codes,
+                           k_scale, k_mean, workspace, stream=None):
+    """sage_quant_qk on projection outputs: QK RMSNorm (BF16 weights [D], eps)
+    and RoPE (float32 cos / sin tables [N, D/2]) applied in the same kernels."""
+    nr = SageNormRope(_ptr(q_weight), _ptr(k_weight), _ptr(rope_cos), _ptr(rope_sin), float(eps))
+    ws_bytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
+    _ok(_lib.sage_quant_qk_normrope(_ptr(q), _ptr(k), shape, ctypes.byref(nr), _ptr(q_codes), _ptr(q_scale),
+                                    _ptr(k_codes), _ptr(k_scale), _ptr(k_mean), _ptr(workspace), ws_bytes,
+                                    _stream(stream)),
+        "sage_quant_qk_normrope")
+
+
 def sage_quant_v(v, shape, v_codes_t, v_scale, v_mean, workspace, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
     _ok(_lib.sage_quant_v(_ptr(v), shape, _ptr(v_codes_t), _ptr(v_scale), _ptr(v_mean), _ptr(workspace),
@@ -189,11 +209,19 @@ class Buffers:
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if with_lse else None
         self.workspace = torch.empty(max(256, workspace_bytes(self.shape)), dtype=torch.uint8, device=dev)
 
-    def run(self, q, k, v, sm_scale=0.0, stream=None, v_shape=None):
+    def run(self, q, k, v, sm_scale=0.0, stream=None, v_shape=None, normrope=None):
         """quant_qk -> quant_v -> attn_fwd; q, k, v are BF16 [B, N, H, D] device tensors
-        (v may be a token-strided view; pass v_shape with its tok_stride)."""
-        sage_quant_qk(q, k, self.shape, self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.k_mean,
-                      self.workspace, stream)
+        (v may be a token-strided view; pass v_shape with its tok_stride).  normrope:
+        None, or dict(q_w, k_w, cos, sin, eps) of device tensors (and a float): Q and K
+        are then projection outputs, normed and rotated inside the quantization."""
+        if normrope is None:
+            sage_quant_qk(q, k, self.shape, self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.k_mean,
+                          self.workspace, stream)
+        else:
+            nr = normrope
+            sage_quant_qk_normrope(q, k, self.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
+                                   self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.k_mean,
+                                   self.workspace, stream)
         sage_quant_v(v, v_shape or self.shape, self.v_codes_t, self.v_scale, self.v_mean, self.workspace, stream)
         sage_attn_fwd(self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.v_codes_t, self.v_scale,
                       self.v_mean, self.shape, sm_scale, self.out, self.out_fp32, self.lse, stream)

@@ -232,19 +232,22 @@ void build_seg_table(const sage_shape& s, sage::SegTable* tab) {
 }
 
 // The INT8 code pass of sage_quant_qk: the 64-token block kernel when both
-// tensors use blocks, the group kernel otherwise.
+// tensors use blocks, the group kernel otherwise.  kNR: rows first go through
+// QK RMSNorm + RoPE (sage_quant_qk_normrope).
+template <bool kNR>
 void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const uint16_t* kb,
                      const uint16_t* kmean, int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale,
-                     cudaStream_t cs) {
+                     const sage::NormRopeArgs& nr, cudaStream_t cs) {
   const int Npad = static_cast<int>(npad_of(s.N));
   if (s.q_gran == SAGE_GRAN_BLOCK64 && s.k_gran == SAGE_GRAN_BLOCK64) {
-    const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
+    // one 128-token tile per CTA, or one 64-token block with the norm / RoPE
+    const dim3 g(Npad / (kNR ? sage::kQKBlock : sage::kTile), s.H, 2 * s.B);
     if (s.D == 128)
-      sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
-                                                   k_codes, k_scale);
+      sage::qk_block_quant<128, kNR><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+                                                        k_codes, k_scale, nr);
     else
-      sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
-                                                  k_codes, k_scale);
+      sage::qk_block_quant<64, kNR><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+                                                       k_codes, k_scale, nr);
     return;
   }
   sage::SegTable tab;
@@ -254,17 +257,19 @@ void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const 
   int gx = 0;
   for (const int g : {s.q_gran, s.k_gran}) gx = std::max(gx, g == SAGE_GRAN_SEGMENT64 ? seg_ctas : tiles);
   const dim3 grid(gx, s.H, 2 * s.B);
-  // The nine (Q, K) granularity pairs, each for D = 64 and 128 (both block64:
-  // qk_block_quant above).
+  // The eight (Q, K) granularity pairs other than (block, block), each for
+  // D = 64 and 128.
   auto launch = [&](auto dq, auto dk) {
     constexpr int GQ = decltype(dq)::value;
     constexpr int GK = decltype(dk)::value;
-    if (s.D == 128)
-      sage::qk_group_quant<128, GQ, GK><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
-                                                              q_scale, k_codes, k_scale, tab);
-    else
-      sage::qk_group_quant<64, GQ, GK><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
-                                                             q_scale, k_codes, k_scale, tab);
+    if constexpr (GQ != sage::kGranBlock64 || GK != sage::kGranBlock64) {
+      if (s.D == 128)
+        sage::qk_group_quant<128, GQ, GK, kNR><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                                                                     q_scale, k_codes, k_scale, tab, nr);
+      else
+        sage::qk_group_quant<64, GQ, GK, kNR><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                                                                    q_scale, k_codes, k_scale, tab, nr);
+    }
   };
   using G0 = std::integral_constant<int, sage::kGranBlock64>;
   using G1 = std::integral_constant<int, sage::kGranToken>;
@@ -369,8 +374,59 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  launch_qk_codes(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, cs);
+  launch_qk_codes<false>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, sage::NormRopeArgs{}, cs);
   return launch_check("sage_quant_qk launch");
+}
+
+sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s, const sage_normrope* nr,
+                                   int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale, void* k_mean,
+                                   void* workspace, size_t ws_bytes, sage_stream_t stream) {
+  int64_t ts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  SAGE_NEED(q, "q");
+  SAGE_NEED(k, "k");
+  SAGE_NEED(q_codes, "q_codes");
+  SAGE_NEED(q_scale, "q_scale");
+  SAGE_NEED(k_codes, "k_codes");
+  SAGE_NEED(k_scale, "k_scale");
+  if (!nr) return fail(SAGE_ERR_INVALID_ARG, "nr is NULL");
+  SAGE_NEED(nr->q_weight, "nr->q_weight");
+  SAGE_NEED(nr->k_weight, "nr->k_weight");
+  SAGE_NEED(nr->rope_cos, "nr->rope_cos");
+  SAGE_NEED(nr->rope_sin, "nr->rope_sin");
+  if (!(nr->eps > 0.f) || !(nr->eps < 3.0e38f)) return fail(SAGE_ERR_INVALID_ARG, "nr->eps must be finite and > 0");
+  if (k_mean && !aligned16(k_mean)) return fail(SAGE_ERR_ALIGNMENT, "k_mean is not 16-byte aligned");
+  WsLayout lay;
+  if ((st = check_ws(s, workspace, ws_bytes, &lay)) != SAGE_OK) return st;
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* psum = reinterpret_cast<double*>(ws + lay.psum);
+  uint16_t* kmean = reinterpret_cast<uint16_t*>(ws + lay.kmean);
+  const int HD = s.H * s.D;
+  const int nsb = (s.N + sage::kSumBlock - 1) / sage::kSumBlock;
+  const uint16_t* qb = static_cast<const uint16_t*>(q);
+  const uint16_t* kb = static_cast<const uint16_t*>(k);
+  sage::NormRopeArgs a;
+  a.q_w = static_cast<const uint16_t*>(nr->q_weight);
+  a.k_w = static_cast<const uint16_t*>(nr->k_weight);
+  a.cos = nr->rope_cos;
+  a.sin = nr->rope_sin;
+  a.eps = nr->eps;
+
+  const dim3 sg(nsb, s.B, (HD + 1023) / 1024);
+  if (s.D == 128)
+    sage::colstats_normrope<128><<<sg, 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum, a);
+  else
+    sage::colstats_normrope<64><<<sg, 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum, a);
+  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
+                                                                static_cast<uint16_t*>(k_mean));
+  launch_qk_codes<true>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, a, cs);
+  return launch_check("sage_quant_qk_normrope launch");
 }
 
 sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t, float* v_scale, float* v_mean,
@@ -548,7 +604,7 @@ sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int
                                                                                     nullptr, nullptr);
   sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
                                                                 static_cast<uint16_t*>(k_mean));
-  launch_qk_codes(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, cs);
+  launch_qk_codes<false>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, sage::NormRopeArgs{}, cs);
   return launch_check("sage_quant_qk_static launch");
 }
 

@@ -40,6 +40,112 @@ __device__ __forceinline__ void unpack8(const uint4& raw, float (&f)[8]) {
 }
 
 // ----------------------------------------------------------------------------
+// QK RMSNorm + RoPE in BF16 rounding, applied to a token row as it is loaded
+// (sage_quant_qk_normrope).  The D channels of one (token, head) row are held
+// by L = D/8 consecutive lanes, 8 channels each.
+//   ss = sum of x^2: each lane adds its 8 squares in order from +0 (x^2 of a
+//        BF16 value is exact, so fma(x, x, ss) is one rounding of ss + x^2),
+//        then ss <- ss + ss[lane ^ o] for o = L/2 .. 1 (every lane ends equal);
+//   r  = RN(1 / RN(sqrt(RN(RN(ss / D) + eps))))   (correctly rounded sqrt, div);
+//   y  = RN_bf16(RN(x * r));  z = RN_bf16(y * w);
+//   pair (z[2i], z[2i+1]) = (a, b) of table pair p = (d0 + 2i) / 2:
+//   o0 = RN_bf16(RN(RN(c * a) - RN(s * b))), o1 = RN_bf16(RN(RN(s * a) + RN(c * b))).
+// ----------------------------------------------------------------------------
+struct NormRopeArgs {
+  const uint16_t* q_w;    // BF16 [D] RMSNorm weight of Q
+  const uint16_t* k_w;    // BF16 [D] RMSNorm weight of K
+  const float* cos;       // [N, D/2] per token and channel pair
+  const float* sin;       // [N, D/2]
+  float eps;
+};
+
+__device__ __forceinline__ f32x2_t x2_of(float lo, float hi) {
+  return x2_pack(__float_as_uint(lo), __float_as_uint(hi));
+}
+
+// RN_bf16 of both halves (one packed conversion), returned as binary32.
+__device__ __forceinline__ f32x2_t x2_bf16_round(f32x2_t v) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x2_lo(v), x2_hi(v));
+  return x2_of(__low2float(b), __high2float(b));
+}
+
+// Both halves RN_bf16, packed (low half = lo).
+__device__ __forceinline__ uint32_t bf16x2_round(f32x2_t v) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x2_hi(v)), "f"(x2_lo(v)));
+  return d;
+}
+
+// RN_bf16(a * b) per half of two packed BF16 pairs (the product of two BF16
+// values is exact, so this is the binary32 product rounded once to BF16).
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// kRows token rows of this lane (8 channels d0 .. d0+7 each), in place.  The
+// kL = D/8 lanes of a row are consecutive lanes of the warp, and every lane of
+// the warp executes this call.  Rows past the data hold zeros and stay zero.
+// The root and reciprocal of row t are formed once, by lane t of the row's
+// lanes, and shuffled out.  cs[t], sn[t]: cos / sin of row t's pairs
+// d0/2 .. d0/2+3.  Products run in f32x2 pairs: the rotation of pair (a, b)
+// is (c*a, s*a) + (-s*b, c*b), each product rounded, then one rounded add per
+// half (RN(-(s*b)) = -RN(s*b), so the first half is RN(RN(c*a) - RN(s*b))).
+template <int kRows, int kL>
+__device__ __forceinline__ void norm_rope_rows(float (&x)[kRows][8], const float (&w)[8], float eps,
+                                               const float4 (&cs)[kRows], const float4 (&sn)[kRows]) {
+  static_assert(kRows <= kL, "one lane per row for the root");
+  constexpr float kInvD = 1.f / static_cast<float>(8 * kL);
+  float ss[kRows];
+#pragma unroll
+  for (int t = 0; t < kRows; ++t) {
+    ss[t] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss[t] = __fmaf_rn(x[t][i], x[t][i], ss[t]);
+  }
+#pragma unroll
+  for (int o = kL / 2; o >= 1; o >>= 1) {
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) ss[t] = __fadd_rn(ss[t], __shfl_xor_sync(0xFFFFFFFFu, ss[t], o));
+  }
+  const int lane = threadIdx.x & 31;
+  const int g = (lane % kL) % kRows;
+  float mine = ss[0];
+#pragma unroll
+  for (int t = 1; t < kRows; ++t) mine = g == t ? ss[t] : mine;
+  const float rl = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fmul_rn(mine, kInvD), eps)));
+  const int base = lane & ~(kL - 1);
+  uint32_t w2[4];                         // the weight pairs as packed BF16 (exact: w is BF16)
+#pragma unroll
+  for (int p = 0; p < 4; ++p) w2[p] = bf16x2_round(x2_of(w[2 * p], w[2 * p + 1]));
+#pragma unroll
+  for (int t = 0; t < kRows; ++t) {
+    const f32x2_t r2 = x2_splat(__shfl_sync(0xFFFFFFFFu, rl, base + t));
+    const float c[4] = {cs[t].x, cs[t].y, cs[t].z, cs[t].w};
+    const float s[4] = {sn[t].x, sn[t].y, sn[t].z, sn[t].w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t y = bf16x2_round(x2_mul(x2_of(x[t][2 * p], x[t][2 * p + 1]), r2));
+      const uint32_t zb = bf16x2_mul(y, w2[p]);
+      const f32x2_t z = x2_of(__uint_as_float(zb << 16), __uint_as_float(zb & 0xFFFF0000u));
+      const f32x2_t t1 = x2_mul(x2_of(c[p], s[p]), x2_splat(x2_lo(z)));
+      const f32x2_t t2 = x2_mul(x2_of(-s[p], c[p]), x2_splat(x2_hi(z)));
+      // Scalar adds: the compiler fuses an f32x2 multiply into a following
+      // f32x2 add (one rounding fewer), but never a product into __fadd_rn.
+      const f32x2_t o = x2_bf16_round(x2_of(__fadd_rn(x2_lo(t1), x2_lo(t2)), __fadd_rn(x2_hi(t1), x2_hi(t2))));
+      x[t][2 * p] = x2_lo(o);
+      x[t][2 * p + 1] = x2_hi(o);
+    }
+  }
+}
+
+__device__ __forceinline__ float4 ld_nc_f4(const float* p) {
+  const uint4 r = ld_nc_16(p);
+  return make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), __uint_as_float(r.w));
+}
+
+// ----------------------------------------------------------------------------
 // Per (b, 64-token block c, channel): s = ((0 + x_{64c}) + x_{64c+1}) + ... in
 // token order, in FP64.  Grid (nsb, B, ceil(HD / (8*blockDim))).
 // ----------------------------------------------------------------------------
@@ -101,6 +207,58 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
     px[0] = make_float4(__low2float(mx[0]), __high2float(mx[0]), __low2float(mx[1]), __high2float(mx[1]));
     px[1] = make_float4(__low2float(mx[2]), __high2float(mx[2]), __low2float(mx[3]), __high2float(mx[3]));
   }
+}
+
+// K column sums (as colstats_partial<false>: same grid, order and output) of
+// the rows after QK RMSNorm + RoPE, for the K mean of sage_quant_qk_normrope.
+// Lanes past H*D run the loop on zeros (their whole head is past it) so that
+// every lane takes part in the row shuffles.
+template <int D>
+__global__ void __launch_bounds__(128) colstats_normrope(const uint16_t* __restrict__ x, int N, int HD,
+                                                         int64_t tok_stride, int nsb, double* __restrict__ psum,
+                                                         const NormRopeArgs nr) {
+  const int c = blockIdx.x;
+  const int b = blockIdx.y;
+  const int ch0 = (blockIdx.z * blockDim.x + threadIdx.x) * 8;
+  const bool active = ch0 < HD;
+  const int d0 = ch0 % D;
+  float w[8];
+  unpack8(active ? ld_nc_16(nr.k_w + d0) : make_uint4(0u, 0u, 0u, 0u), w);
+  const int n0 = c * kSumBlock;
+  const int n1 = min(N, n0 + kSumBlock);
+  const uint16_t* p = x + (static_cast<int64_t>(b) * N + n0) * tok_stride + (active ? ch0 : 0);
+  double s[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s[i] = 0.0;
+  constexpr int kRows = 4;                 // rows (and their table entries) in flight
+  for (int n = n0; n < n1; n += kRows) {
+    uint4 raw[kRows];
+    float4 cs[kRows], sn[kRows];
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) {
+      const bool ok = active && n + t < n1;
+      const int64_t tab = static_cast<int64_t>(n + t) * (D / 2) + d0 / 2;
+      raw[t] = ok ? ld_nc_16(p + static_cast<int64_t>(n + t - n0) * tok_stride) : make_uint4(0u, 0u, 0u, 0u);
+      cs[t] = ok ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+      sn[t] = ok ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float f[kRows][8];
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) unpack8(raw[t], f[t]);
+    norm_rope_rows<kRows, D / 8>(f, w, nr.eps, cs, sn);
+#pragma unroll
+    for (int t = 0; t < kRows; ++t) {
+      if (n + t < n1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] = __dadd_rn(s[i], static_cast<double>(f[t][i]));
+      }
+    }
+  }
+  if (!active) return;
+  const int64_t o = (static_cast<int64_t>(b) * nsb + c) * HD + ch0;
+  double2* ps = reinterpret_cast<double2*>(psum + o);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ps[i] = make_double2(s[2 * i], s[2 * i + 1]);
 }
 
 // Second level of the fixed summation order for one channel: lane g sums
@@ -224,19 +382,25 @@ __device__ __forceinline__ int rne_small(float y) {
   return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
 }
 
-template <int D>
-__global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict__ q,
+// kNR: Q and K rows first go through QK RMSNorm + RoPE (norm_rope_rows); that
+// variant takes one 64-token block per CTA (4 rows per thread), so that two
+// CTAs fit an SM and one's loads overlap the other's reduction and stores.
+template <int D, bool kNR = false>
+__global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_t* __restrict__ q,
                                                       const uint16_t* __restrict__ k, int N, int B, int H,
                                                       int Npad, int64_t tok_stride,
                                                       const uint16_t* __restrict__ k_mean,
                                                       int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
                                                       int8_t* __restrict__ k_codes,
-                                                      float* __restrict__ k_scale) {
+                                                      float* __restrict__ k_scale, const NormRopeArgs nr = {}) {
+  constexpr int kWarps = 256 / 32;
+  constexpr int kSlots = kNR ? 1 : 2;     // 64-token blocks per CTA
+  constexpr int kTokens = kSlots * kQKBlock;
   constexpr int kLPR = D / 8;             // threads per token row
   constexpr int kRPP = 256 / kLPR;        // token rows per pass
-  constexpr int kTPT = kTile / kRPP;      // tokens per thread (half in each 64-token block)
-  constexpr int kHalf = kTPT / 2;
-  __shared__ float red[8][2];
+  constexpr int kTPT = kTokens / kRPP;    // tokens per thread (kHalf in each block)
+  constexpr int kHalf = kTPT / kSlots;
+  __shared__ float red[kWarps][2];
   const int tile = blockIdx.x;
   const bool is_k = static_cast<int>(blockIdx.z) < B;
   // K heads are visited last-to-first: the column-sum pass just streamed K in
@@ -254,18 +418,30 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
     unpack8(mraw, mean);
   }
   uint4 raw[kTPT];
+  float4 cs[kNR ? kTPT : 1], sn[kNR ? kTPT : 1];
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
-    const int n = tile * kTile + r0 + t * kRPP;
+    const int n = tile * kTokens + r0 + t * kRPP;
     raw[t] = n < N ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
                    : make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (kNR) {
+      const int64_t tab = static_cast<int64_t>(n) * (D / 2) + d0 / 2;
+      cs[t] = n < N ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+      sn[t] = n < N ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   float x[kTPT][8];
   float amax[2] = {0.f, 0.f};
 #pragma unroll
+  for (int t = 0; t < kTPT; ++t) unpack8(raw[t], x[t]);
+  if constexpr (kNR) {
+    float nw[8];
+    unpack8(ld_nc_16((is_k ? nr.k_w : nr.q_w) + d0), nw);
+    norm_rope_rows<kTPT, kLPR>(x, nw, nr.eps, cs, sn);   // rows past N stay zero
+  }
+#pragma unroll
   for (int t = 0; t < kTPT; ++t) {
-    const int n = tile * kTile + r0 + t * kRPP;
-    unpack8(raw[t], x[t]);
+    const int n = tile * kTokens + r0 + t * kRPP;
     if (is_k) {
       if (n < N) {
 #pragma unroll
@@ -295,7 +471,7 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
   for (int blk = 0; blk < 2; ++blk) {
     float a = red[0][blk];
 #pragma unroll
-    for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w][blk]);
+    for (int w = 1; w < kWarps; ++w) a = fmaxf(a, red[w][blk]);
     scale[blk] = 0.f;
     inv[blk] = 0.f;
     if (a > 0.f) {
@@ -307,7 +483,7 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
   int8_t* dst = is_k ? k_codes : q_codes;
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
-    const int n = tile * kTile + r0 + t * kRPP;
+    const int n = tile * kTokens + r0 + t * kRPP;
     const float iv = inv[t / kHalf];
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -318,7 +494,8 @@ __global__ void __launch_bounds__(256) qk_block_quant(const uint16_t* __restrict
     }
     *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w[0], w[1]);
   }
-  if (threadIdx.x < 2) (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + tile * 2 + threadIdx.x] = scale[threadIdx.x];
+  if (threadIdx.x < kSlots)
+    (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + tile * kSlots + threadIdx.x] = threadIdx.x == 0 ? scale[0] : scale[1];
 }
 
 // ----------------------------------------------------------------------------
@@ -357,13 +534,13 @@ __device__ __forceinline__ void seg_block(const SegTable& seg, int g, int& start
 }
 
 // One CTA of qk_group_quant: tensor K (is_k) or Q at granularity kGran.
-template <int D, int kGran>
+template <int D, int kGran, bool kNR>
 __device__ __forceinline__ void group_quant_cta(bool is_k, const uint16_t* __restrict__ q,
                                                 const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
                                                 int64_t tok_stride, const uint16_t* __restrict__ k_mean,
                                                 int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
                                                 int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
-                                                const SegTable& seg) {
+                                                const SegTable& seg, const NormRopeArgs& nr) {
   constexpr int gran = kGran;
   constexpr int kLPR = D / 8;             // threads per token row
   constexpr int kRPP = 256 / kLPR;        // token rows per pass
@@ -403,21 +580,33 @@ __device__ __forceinline__ void group_quant_cta(bool is_k, const uint16_t* __res
     unpack8(mraw, mean);
   }
   uint4 raw[kTPT];
+  float4 cs[kNR ? kTPT : 1], sn[kNR ? kTPT : 1];
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
     const int o = r0 + (t % kHalf) * kRPP;
     const int n = gstart[t / kHalf] + o;
-    raw[t] = (o < glen[t / kHalf] && n < N)
-                 ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
-                 : make_uint4(0u, 0u, 0u, 0u);
+    const bool ok = o < glen[t / kHalf] && n < N;
+    raw[t] = ok ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
+                : make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (kNR) {
+      const int64_t tab = static_cast<int64_t>(n) * (D / 2) + d0 / 2;
+      cs[t] = ok ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+      sn[t] = ok ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   float x[kTPT][8];
   float rmax[kTPT];
 #pragma unroll
+  for (int t = 0; t < kTPT; ++t) unpack8(raw[t], x[t]);
+  if constexpr (kNR) {
+    float nw[8];
+    unpack8(ld_nc_16((is_k ? nr.k_w : nr.q_w) + d0), nw);
+    norm_rope_rows<kTPT, kLPR>(x, nw, nr.eps, cs, sn);   // rows not loaded stay zero
+  }
+#pragma unroll
   for (int t = 0; t < kTPT; ++t) {
     const int o = r0 + (t % kHalf) * kRPP;
     const int n = gstart[t / kHalf] + o;
-    unpack8(raw[t], x[t]);
     if (is_k && o < glen[t / kHalf] && n < N) {
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
@@ -520,18 +709,18 @@ __device__ __forceinline__ void group_quant_cta(bool is_k, const uint16_t* __res
 
 // Grid (max CTAs of the two tensors, H, 2B): z < B quantizes K at kGranK, the
 // rest Q at kGranQ.  A CTA past its tensor's tiles or blocks leaves at once.
-template <int D, int kGranQ, int kGranK>
-__global__ void __launch_bounds__(256, (kGranQ == kGranSegment64 || kGranK == kGranSegment64) ? 2 : 3)
+template <int D, int kGranQ, int kGranK, bool kNR = false>
+__global__ void __launch_bounds__(256, kNR ? 1 : ((kGranQ == kGranSegment64 || kGranK == kGranSegment64) ? 2 : 3))
     qk_group_quant(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
                    int64_t tok_stride, const uint16_t* __restrict__ k_mean, int8_t* __restrict__ q_codes,
                    float* __restrict__ q_scale, int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
-                   const __grid_constant__ SegTable seg) {
+                   const __grid_constant__ SegTable seg, const NormRopeArgs nr = {}) {
   if (static_cast<int>(blockIdx.z) < B)
-    group_quant_cta<D, kGranK>(true, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes, k_scale,
-                               seg);
+    group_quant_cta<D, kGranK, kNR>(true, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes,
+                                    k_scale, seg, nr);
   else
-    group_quant_cta<D, kGranQ>(false, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes,
-                               k_scale, seg);
+    group_quant_cta<D, kGranQ, kNR>(false, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes,
+                                    k_scale, seg, nr);
 }
 
 // ----------------------------------------------------------------------------

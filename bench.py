@@ -85,6 +85,8 @@ def parse():
                     help="INT8 scale groups of Q (default: 64-token blocks)")
     ap.add_argument("--k-gran", default="block64", choices=["block64", "token", "segment64"],
                     help="INT8 scale groups of K (default: 64-token blocks)")
+    ap.add_argument("--normrope", action="store_true",
+                    help="Q and K are projection outputs: QK RMSNorm + RoPE fused into the quantization")
     ap.add_argument("--peaks", action="store_true",
                     help="measure library INT8 / FP8 / BF16 GEMM throughput at 8192^3 and exit")
     return ap.parse_args()
@@ -180,13 +182,13 @@ def gpu_id_for(dev_index: int):
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_sample(w, qb, kb, vb, rows: int, heads: int, q_gran="block64", k_gran="block64"):
+def oracle_sample(w, qb, kb, vb, rows: int, heads: int, q_gran="block64", k_gran="block64", normrope=None):
     """Time the CPU oracle on `heads` heads of batch 0 (full quantization of those
     heads, attention for `rows` query rows).  Returns (ops, seconds)."""
     from oracle import sage_oracle as so
     t0 = time.perf_counter()
     sl = (slice(0, 1), slice(None), slice(0, heads), slice(None))
-    qk = so.quant_qk(qb[sl], kb[sl], q_gran, k_gran, w.cu_seqlens)
+    qk = so.quant_qk(qb[sl], kb[sl], q_gran, k_gran, w.cu_seqlens, normrope=normrope)
     vv = so.quant_v(vb[sl])
     r = synth.sample_rows(w.N, rows, 0)[:rows] if rows < w.N else None
     so.attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"], vv["v_codes_t"], vv["v_scale"],
@@ -294,15 +296,28 @@ def main():
                                 device_id=torch.device("cuda", local))
     w = synth.WORKLOADS[args.workload]
     qb, kb, vb = synth.generate(w)
+    nr_host = None
+    if args.normrope:
+        qb, kb = synth.projection_outputs(w)
+        nr_host = synth.normrope_inputs(w)
     as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
     q, k, v = as_dev(qb), as_dev(kb), as_dev(vb)
+    nr = None
+    if nr_host is not None:
+        nr = dict(q_w=as_dev(nr_host["q_w"]), k_w=as_dev(nr_host["k_w"]), eps=nr_host["eps"],
+                  cos=torch.from_numpy(nr_host["cos"]).cuda(), sin=torch.from_numpy(nr_host["sin"]).cuda())
     buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=args.q_gran, k_gran=args.k_gran)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     def quant_qk():
-        adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                          buf.workspace, stream)
+        if nr is None:
+            adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                              buf.workspace, stream)
+        else:
+            adt.sage_quant_qk_normrope(q, k, buf.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
+                                       buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                                       buf.workspace, stream)
 
     def quant_v():
         adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
@@ -382,12 +397,14 @@ def main():
     attn_mean_ms = statistics.mean(at_ms)
     achieved = ops / (attn_mean_ms / 1e3) / 1e12
     qk_bytes, v_bytes = quant_bytes(w, args.q_gran, args.k_gran)
+    if nr is not None:
+        qk_bytes += w.N * w.D // 2 * 8 + 2 * w.D * 2          # cos / sin tables once, the two weights
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of CPU work on the GPU machine's host: 4 heads, 2^26 (query row, key) pairs
         heads = min(4, w.H)
         rows = max(1, min(w.N, (1 << 26) // (heads * w.N)))
-        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads, args.q_gran, args.k_gran)
+        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads, args.q_gran, args.k_gran, nr_host)
         cpu = {"value": o_ops / o_dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
                "sample": f"{heads} heads of batch 0: full K/V quantization of those heads + attention for "
                          f"{rows} query rows each ({o_dt:.1f} s)"}
@@ -402,7 +419,8 @@ def main():
         "vs_baseline": None, "dtype": "i8/e4m3 (fp32 softmax)", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "global_batch": w.B * world,
                    "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)",
-                   "q_gran": args.q_gran, "k_gran": args.k_gran},
+                   "q_gran": args.q_gran, "k_gran": args.k_gran,
+                   "qk_prologue": "rmsnorm+rope" if nr is not None else None},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": attn_traffic(w.name) if k_blocks else None,
                      "kernel": f"sage_attn_kernel<{w.D}, {'false' if k_blocks else 'true'}>",

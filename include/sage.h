@@ -138,6 +138,43 @@ SAGE_API sage_status sage_quant_qk(const void* q, const void* k, sage_shape s,
                           void* workspace, size_t ws_bytes, sage_stream_t stream);
 
 /*
+ * sage_quant_qk_normrope - sage_quant_qk on Q and K straight from the
+ * projection: each (token, head) row first goes through RMSNorm and the rotary
+ * position embedding, in BF16 rounding, inside the same kernels (the separate
+ * BF16 write and re-read of the normed Q and K are gone).  ("FLUX 3 Action",
+ * 1 Model Introduction: 4-axis (t, h, w, l) RoPE in the joint blocks; its
+ * serving notes: QK RMSNorm + RoPE as one fused kernel at BF16 rounding level;
+ * "FLUX.3 Action RTX 5090 report", last-round card B.)
+ *
+ * in : q, k        BF16 [B, N, H, D] projection outputs, s.tok_stride.
+ *      nr          weights, eps and rotation tables (below); all device
+ *                  pointers 16-byte aligned; eps finite and > 0.
+ * out: as sage_quant_qk (any q_gran / k_gran).
+ * Rule for one row x of D channels (L = D/8 lanes of 8 channels):
+ *   ss = FP32 sum of x^2: lane g adds channels 8g .. 8g+7 in order from +0,
+ *        then ss_g <- ss_g + ss_{g xor o} for o = L/2 .. 1;
+ *   r  = RN(1 / RN(sqrt(RN(RN(ss / D) + eps))))  (correctly rounded);
+ *   z  = RN_bf16(RN_bf16(RN(x * r)) * w);
+ *   pair i = (z[2i], z[2i+1]) = (a, b), c = rope_cos[n, i], s = rope_sin[n, i]:
+ *   out[2i] = RN_bf16(RN(RN(c*a) - RN(s*b))), out[2i+1] = RN_bf16(RN(RN(s*a) + RN(c*b))).
+ * The K mean, K centring and INT8 rule of sage_quant_qk then apply to the
+ * rows so produced.  Codes are bit-exact with that rule.
+ */
+typedef struct {
+  const void* q_weight;    /* BF16 [D] RMSNorm weight of Q                    */
+  const void* k_weight;    /* BF16 [D] RMSNorm weight of K                    */
+  const float* rope_cos;   /* f32 [N, D/2]: cos of token n's angle for pair i  */
+  const float* rope_sin;   /* f32 [N, D/2]: its sine                           */
+  float eps;               /* added to the mean square, > 0                    */
+} sage_normrope;
+
+SAGE_API sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s,
+                                            const sage_normrope* nr,
+                                            int8_t* q_codes, float* q_scale,
+                                            int8_t* k_codes, float* k_scale, void* k_mean,
+                                            void* workspace, size_t ws_bytes, sage_stream_t stream);
+
+/*
  * sage_quant_v - V smoothing and per-channel FP8 E4M3 quantization, written
  * transposed.  ("FLUX.3 Action RTX 5090 report", last-round card C; card 03.)
  *

@@ -112,3 +112,26 @@ def test_attn_and_v_validation(adt):
     assert L.sage_quant_v(FAKE, adt.make_shape(1, 256, 2, 128, 200), FAKE, FAKE, FAKE, 0x100000, 1 << 40,
                           None) == 1
     assert L.sage_selftest_wait_timeout(0, None) == 1
+
+
+def test_normrope_validation(adt):
+    L = adt._lib
+    s = adt.make_shape(1, 256, 2, 64)
+
+    def call(nr, **over):
+        a = dict(q=FAKE, k=FAKE, qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE)
+        a.update(over)
+        ref = ctypes.byref(nr) if nr is not None else None
+        return L.sage_quant_qk_normrope(a["q"], a["k"], s, ref, a["qc"], a["qs"], a["kc"], a["ks"], None,
+                                        0x100000, 1 << 40, None)
+
+    good = dict(q_weight=FAKE, k_weight=FAKE, rope_cos=FAKE, rope_sin=FAKE, eps=1e-6)
+    assert call(None) == 1
+    assert call(adt.SageNormRope(**dict(good, q_weight=None))) == 1
+    assert call(adt.SageNormRope(**dict(good, rope_sin=FAKE + 4))) == 3
+    for eps in (0.0, -1e-6, float("inf"), float("nan")):
+        assert call(adt.SageNormRope(**dict(good, eps=eps))) == 1
+        assert b"eps" in L.sage_last_error()
+    assert call(adt.SageNormRope(**good), q=None) == 1
+    if not _gpu_present():
+        assert call(adt.SageNormRope(**good)) == 4

@@ -167,3 +167,20 @@ def test_quant_qk_with_normrope_is_quant_of_the_normed_rotated_bf16():
     again = so.quant_qk(synth.to_bf16_bits(qf), k, normrope=dict(inp, eps=0.0))
     ref = so.quant_qk(q, k, normrope=dict(inp, eps=0.0))
     assert np.array_equal(again["q_codes"], ref["q_codes"])
+
+
+def test_parity_case_can_tell_a_fused_rotation_apart():
+    """The D = 128 GPU parity case holds rotations that land within an ulp of a
+    BF16 midpoint, where RN(RN(c*a) - RN(s*b)) and a fused multiply-add
+    (RN(c*a - RN(s*b)), one rounding fewer) round to different BF16 values, so
+    that case would catch a kernel whose rotation got fused."""
+    w = synth.custom(2, 1000, 3, 128, seed=1500, k_sigma=4.0, v_sigma=1.0, outlier_frac=0.02)
+    q, _ = synth.projection_outputs(w)
+    inp = synth.normrope_inputs(w)
+    z = _f(nr.rms_norm_bf16(q, inp["q_w"], inp["eps"])).astype(np.float64)
+    c = inp["cos"][None, :, None, :].astype(np.float64)
+    s = inp["sin"][None, :, None, :].astype(np.float64)
+    a, b = z[..., 0::2], z[..., 1::2]
+    sep = (np.float32(c * a) - np.float32(s * b)).astype(np.float32)
+    fused = (c * a - np.float32(s * b).astype(np.float64)).astype(np.float32)
+    assert np.count_nonzero(_bf(sep) != _bf(fused)) >= 1
