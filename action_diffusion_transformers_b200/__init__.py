@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
                 4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_DEVICE_TIMEOUT", 6: "SAGE_ERR_WORKSPACE"}
 EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
             "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error",
-            "sage_quant_qk_static", "sage_quant_qk_normrope")
+            "sage_quant_qk_static", "sage_quant_qk_normrope", "sage_fp8_quant_rows", "sage_fp8_linear")
 QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -62,6 +62,11 @@ _lib.sage_quant_qk_static.restype = ctypes.c_int
 _lib.sage_quant_qk_normrope.argtypes = [_vp, _vp, SageShape, ctypes.POINTER(SageNormRope), _vp, _vp, _vp, _vp, _vp,
                                         _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_qk_normrope.restype = ctypes.c_int
+_lib.sage_fp8_quant_rows.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
+_lib.sage_fp8_quant_rows.restype = ctypes.c_int
+_lib.sage_fp8_linear.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int,
+                                 _vp]
+_lib.sage_fp8_linear.restype = ctypes.c_int
 _lib.sage_quant_v.argtypes = [_vp, SageShape, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_v.restype = ctypes.c_int
 _lib.sage_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, SageShape, ctypes.c_float, _vp, ctypes.c_int,
@@ -155,6 +160,23 @@ def sage_quant_qk_normrope(q, k, shape, q_weight, k_weight, rope_cos, rope_sin, 
                                     _ptr(k_codes), _ptr(k_scale), _ptr(k_mean), _ptr(workspace), ws_bytes,
                                     _stream(stream)),
         "sage_quant_qk_normrope")
+
+
+def sage_fp8_quant_rows(x, codes, scale, stream=None):
+    """Per-row E4M3 codes [R, K] (uint8) and scales [R] (float32) of a BF16 [R, K]
+    tensor whose rows may be strided (x.stride(1) must be 1)."""
+    R, K = x.shape
+    assert x.stride(1) == 1
+    _ok(_lib.sage_fp8_quant_rows(_ptr(x), R, K, x.stride(0), _ptr(codes), _ptr(scale), _stream(stream)),
+        "sage_fp8_quant_rows")
+
+
+def sage_fp8_linear(xq, sx, wq, sw, out, stream=None):
+    """out [M, N] (BF16 or float32) = row-wise FP8 product of xq [M, K] and wq [N, K]."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    _ok(_lib.sage_fp8_linear(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(out),
+                             1 if out.dtype == torch.float32 else 0, _stream(stream)), "sage_fp8_linear")
 
 
 def sage_quant_v(v, shape, v_codes_t, v_scale, v_mean, workspace, stream=None):

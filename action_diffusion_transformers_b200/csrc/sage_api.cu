@@ -18,6 +18,7 @@
 #include <type_traits>
 
 #include "sage.h"
+#include "fp8_linear.cuh"
 #include "sage_attn.cuh"
 #include "sage_quant.cuh"
 
@@ -97,6 +98,9 @@ sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullpt
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(sage::sage_attn_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::AttnSmem<64>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::GemmSmem::kAlloc);
       if (e == cudaSuccess && !g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -531,6 +535,69 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   else
     sage::sage_attn_kernel<64, true><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
   return launch_check("sage_attn_fwd launch");
+}
+
+sage_status sage_fp8_quant_rows(const void* x, int R, int K, int64_t ld, uint8_t* codes, float* scale,
+                                sage_stream_t stream) {
+  if (R < 1 || K < 8) return fail(SAGE_ERR_INVALID_ARG, "R >= 1 and K >= 8 required (got %d, %d)", R, K);
+  if (K % 8 != 0) return fail(SAGE_ERR_ALIGNMENT, "K = %d is not a multiple of 8", K);
+  if (K > 16384) return fail(SAGE_ERR_UNSUPPORTED, "K = %d above 16384", K);
+  const int64_t lds = ld == 0 ? K : ld;
+  if (lds < K || lds % 8 != 0) return fail(SAGE_ERR_ALIGNMENT, "ld = %lld must be >= K and a multiple of 8", (long long)lds);
+  SAGE_NEED(x, "x");
+  SAGE_NEED(codes, "codes");
+  if (!scale) return fail(SAGE_ERR_INVALID_ARG, "scale is NULL");
+  if (reinterpret_cast<uintptr_t>(scale) & 3u) return fail(SAGE_ERR_ALIGNMENT, "scale is not 4-byte aligned");
+  int dev;
+  int* err;
+  sage_status st;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  const int per = K / 8;
+  if (per <= 4 * sage::kFqThreads)
+    sage::fp8_quant_rows_kernel<4><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+  else if (per <= 8 * sage::kFqThreads)
+    sage::fp8_quant_rows_kernel<8><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+  else
+    sage::fp8_quant_rows_kernel<16><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+  return launch_check("sage_fp8_quant_rows launch");
+}
+
+sage_status sage_fp8_linear(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw, int M, int N,
+                            int K, void* out, int out_fp32, sage_stream_t stream) {
+  if (M < 1 || N < 1 || K < 16) return fail(SAGE_ERR_INVALID_ARG, "M, N >= 1 and K >= 16 required");
+  if (K % 16 != 0) return fail(SAGE_ERR_ALIGNMENT, "K = %d is not a multiple of 16", K);
+  if (N % 8 != 0) return fail(SAGE_ERR_ALIGNMENT, "N = %d is not a multiple of 8", N);
+  SAGE_NEED(xq, "xq");
+  SAGE_NEED(wq, "wq");
+  SAGE_NEED(sx, "sx");
+  SAGE_NEED(sw, "sw");
+  SAGE_NEED(out, "out");
+  int dev;
+  int* err;
+  int sm_count = 0;
+  sage_status st;
+  if ((st = device_setup(&dev, &err, &sm_count)) != SAGE_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = encode_2d(&ta, xq, K, M, sage::kGemmBK, sage::kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK) return st;
+  if ((st = encode_2d(&tb, wq, K, N, sage::kGemmBK, sage::kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK) return st;
+  sage::GemmParams prm;
+  prm.sx = sx;
+  prm.sw = sw;
+  prm.out = out;
+  prm.M = M;
+  prm.N = N;
+  prm.K = K;
+  prm.out_fp32 = out_fp32 ? 1 : 0;
+  prm.err = err;
+  prm.timeout_ns = g_timeout_ns.load();
+  const int64_t tiles = static_cast<int64_t>((M + sage::kGemmBM - 1) / sage::kGemmBM) *
+                        ((N + sage::kGemmBN - 1) / sage::kGemmBN);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sm_count > 0 ? sm_count : 148));
+  sage::fp8_gemm_kernel<<<grid, sage::kGemmThreads, sage::GemmSmem::kAlloc,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(ta, tb, prm);
+  return launch_check("sage_fp8_linear launch");
 }
 
 sage_status sage_check(sage_stream_t stream) {

@@ -218,6 +218,37 @@ SAGE_API sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale,
                           void* out, int out_fp32, float* lse,
                           sage_stream_t stream);
 
+/*
+ * sage_fp8_quant_rows - per-row E4M3 quantization of a BF16 matrix, for the
+ * activations (one scale per token) and, offline, the weights (one scale per
+ * output row) of sage_fp8_linear.  ("FLUX.3 Action RTX 5090 report", 02
+ * ENGINEERING card 02: E4M3 projections with one scale per output row; "FLUX 3
+ * Action" serving notes: per-token activation scales.)
+ *
+ * in : x       BF16 [R, K], row stride ld elements (0 means K; ld % 8 == 0).
+ * out: codes   E4M3 bytes [R, K] (contiguous); scale f32 [R].
+ * Rule per row: amax = max|x|, scale = RN(amax/448), inv = RN(448/amax),
+ * code = E4M3_RNE_satfinite(RN(x * inv)); amax == 0 gives 0 scale and codes.
+ * K % 8 == 0, 8 <= K <= 16384.  Bit-exact with that rule.
+ */
+SAGE_API sage_status sage_fp8_quant_rows(const void* x, int R, int K, int64_t ld, uint8_t* codes,
+                                         float* scale, sage_stream_t stream);
+
+/*
+ * sage_fp8_linear - y = X W^T with row-wise FP8 operands on the tensor cores.
+ *
+ * in : xq E4M3 [M, K], sx f32 [M] (sage_fp8_quant_rows of the activations);
+ *      wq E4M3 [N, K], sw f32 [N] (the weights' per-row codes and scales).
+ * out: out [M, N] BF16 (out_fp32 == 0) or FP32, row-major.
+ * acc[m, n] = sum_k xq[m,k] * wq[n,k] accumulated in FP32 by the tensor core;
+ * y = RN(RN(acc * sx[m]) * sw[n]); the BF16 output is RN_bf16 of y.
+ * K % 16 == 0, N % 8 == 0; all pointers 16-byte aligned.  The FP32 summation
+ * order is the tensor core's, so results match an exact accumulation within
+ * FP32 rounding, not bit for bit.
+ */
+SAGE_API sage_status sage_fp8_linear(const uint8_t* xq, const float* sx, const uint8_t* wq, const float* sw,
+                                     int M, int N, int K, void* out, int out_fp32, sage_stream_t stream);
+
 /* Synchronises `stream`, then reports and clears a device-side wait timeout
  * raised by any kernel of this library (SAGE_ERR_DEVICE_TIMEOUT), or a CUDA
  * error (SAGE_ERR_CUDA); SAGE_OK otherwise. */

@@ -57,11 +57,18 @@ def _units(codes: np.ndarray) -> np.ndarray:
 
 
 def fp8_accumulate(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
-    """Exact acc[m, n] = sum_k dec(xq[m, k]) * dec(wq[n, k]) as float64 (exact)."""
+    """Exact acc[m, n] = sum_k dec(xq[m, k]) * dec(wq[n, k]) as float64 (exact).
+
+    In units of 2^-18 every product is an integer below 2^36; for K <= 2^17
+    every partial sum stays below 2^53, so a float64 matrix product of the
+    integer units is exact in any summation order; beyond that, int64."""
     a = _units(xq)
     b = _units(wq)
-    acc = a @ b.T                                          # int64, units of 2^-18
-    return acc.astype(np.float64) * 2.0 ** -18
+    if xq.shape[1] <= 1 << 17:
+        acc = a.astype(np.float64) @ b.T.astype(np.float64)
+    else:
+        acc = (a @ b.T).astype(np.float64)
+    return acc * 2.0 ** -18
 
 
 def fp8_linear(xq, sx, wq, sw) -> np.ndarray:

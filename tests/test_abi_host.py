@@ -135,3 +135,17 @@ def test_normrope_validation(adt):
     assert call(adt.SageNormRope(**good), q=None) == 1
     if not _gpu_present():
         assert call(adt.SageNormRope(**good)) == 4
+
+
+def test_fp8_linear_validation(adt):
+    L = adt._lib
+    assert L.sage_fp8_quant_rows(FAKE, 4, 12, 0, FAKE, FAKE, None) == 3      # K % 8
+    assert L.sage_fp8_quant_rows(FAKE, 4, 32768, 0, FAKE, FAKE, None) == 2   # K too large
+    assert L.sage_fp8_quant_rows(FAKE, 4, 64, 60, FAKE, FAKE, None) == 3     # ld < K
+    assert L.sage_fp8_quant_rows(None, 4, 64, 0, FAKE, FAKE, None) == 1
+    assert L.sage_fp8_linear(FAKE, FAKE, FAKE, FAKE, 16, 16, 24, FAKE, 0, None) == 3   # K % 16
+    assert L.sage_fp8_linear(FAKE, FAKE, FAKE, FAKE, 16, 12, 32, FAKE, 0, None) == 3   # N % 8
+    assert L.sage_fp8_linear(FAKE, FAKE, FAKE, FAKE, 0, 16, 32, FAKE, 0, None) == 1
+    assert L.sage_fp8_linear(FAKE, FAKE, FAKE + 4, FAKE, 16, 16, 32, FAKE, 0, None) == 3
+    if not _gpu_present():
+        assert L.sage_fp8_linear(FAKE, FAKE, FAKE, FAKE, 16, 16, 32, FAKE, 0, None) == 4

@@ -80,3 +80,14 @@ def test_linear_power_of_two_identities_and_closed_form():
     yi = fl.fp8_linear(xq, sx, *eye)
     xf = bf16_bits_to_f32(x).astype(np.float64)
     assert np.all(np.abs(yi - xf) <= np.abs(xf) * 2.0 ** -4 + sx[:, None] * 2.0 ** -9 + 1e-7)
+
+
+def test_float64_and_int64_accumulations_agree():
+    rng = np.random.default_rng(5)
+    xq = rng.integers(0, 256, size=(4, 4096), dtype=np.uint8)
+    wq = rng.integers(0, 256, size=(6, 4096), dtype=np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0
+    wq[(wq & 0x7F) == 0x7F] = 0
+    a = fl._units(xq)
+    b = fl._units(wq)
+    assert np.array_equal(fl.fp8_accumulate(xq, wq), (a @ b.T).astype(np.float64) * 2.0 ** -18)
