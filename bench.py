@@ -53,6 +53,26 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def kernel_traffic(key: str, sources, workload: str):
+    """DRAM bytes per launch of a kernel from the last ncu capture of it, if that
+    capture was taken on this workload and on the current kernel source
+    (SHA-256 of `sources`); None otherwise."""
+    import hashlib
+    pkg = os.path.join(ROOT, "action_diffusion_transformers_b200")
+    try:
+        with open(os.path.join(pkg, "ncu_counters.json")) as f:
+            rec = json.load(f)[key]
+    except (OSError, KeyError, ValueError):
+        return None
+    h = hashlib.sha256()
+    for name in sources:
+        with open(os.path.join(pkg, "csrc", name), "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def attn_traffic(workload: str):
     """DRAM bytes per launch of the attention kernel from the last ncu capture,
     if that capture was taken on this workload and on the current kernel source
@@ -85,6 +105,9 @@ def parse():
                     help="INT8 scale groups of Q (default: 64-token blocks)")
     ap.add_argument("--k-gran", default="block64", choices=["block64", "token", "segment64"],
                     help="INT8 scale groups of K (default: 64-token blocks)")
+    ap.add_argument("--op", default="attention", choices=["attention", "fp8_linear"],
+                    help="attention: the quantized attention path (default); fp8_linear: the row-wise "
+                         "FP8 projections of a joint block on the same tokens")
     ap.add_argument("--normrope", action="store_true",
                     help="Q and K are projection outputs: QK RMSNorm + RoPE fused into the quantization")
     ap.add_argument("--peaks", action="store_true",
@@ -207,10 +230,40 @@ def blas_threads():
         return 1
 
 
+def run_reference_fp8(args, w):
+    host = []
+    for i, (name, K, N) in enumerate(fp8_shapes(w)):
+        xb, wb = fp8_inputs(w, K, N, w.seed * 10 + i)
+        host.append((xb, wb, (K, N)))
+    rows = 16
+    for _ in range(args.warmup):
+        fp8_oracle_sample(w, host, rows)
+    times = []
+    flops = 0.0
+    for _ in range(args.steps):
+        flops, dt = fp8_oracle_sample(w, host, rows)
+        times.append(dt)
+    tot = sum(times)
+    value = flops * len(times) / tot / 1e12
+    sample = f"{rows} tokens through each of the {len(host)} projections"
+    line = {"impl": "reference", "metric": "fp8 projection TFLOPS", "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 exact (CPU oracle)", "data": "synthetic",
+            "config": {"workload": f"{w.name} joint-block projections", "tokens": w.B * w.N, "hidden": w.H * w.D},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, rank):
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
+    if args.op == "fp8_linear":
+        run_reference_fp8(args, w)
+        return
     qb, kb, vb = synth.generate(w)
     rows, heads = 256, 1
     grans = (args.q_gran, args.k_gran)
@@ -271,6 +324,176 @@ def measure_peaks(reps: int = 20):
     return out
 
 
+# ----------------------------------------------------------------------------- FP8 projections
+def fp8_shapes(w):
+    """(name, K, N) of the FP8 projections of one joint block on the workload's
+    tokens (hidden H*D, MLP ratio 4): attention output, MLP up, MLP down."""
+    hid = w.H * w.D
+    return [("attn_out", hid, hid), ("mlp_up", hid, 4 * hid), ("mlp_down", 4 * hid, hid)]
+
+
+def fp8_inputs(w, K, N, seed):
+    """Seeded BF16 activations [M, K] (per-token log-normal magnitude) and weights [N, K] ~ N(0, 0.02^2)."""
+    rng = np.random.default_rng(70_000 + seed)
+    M = w.B * w.N
+    x = (rng.standard_normal((M, K), dtype=np.float32) * np.exp(rng.standard_normal((M, 1))).astype(np.float32))
+    wt = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    return synth.to_bf16_bits(x), synth.to_bf16_bits(wt)
+
+
+def fp8_oracle_sample(w, host, rows: int):
+    """The CPU oracle on `rows` tokens of every projection (weights quantized
+    once, outside the timing).  Returns (flops, seconds)."""
+    from oracle import fp8_linear as fl
+    wq = [fl.fp8_quant_rows(wb) for _, wb, _ in host]
+    t0 = time.perf_counter()
+    flops = 0.0
+    for (xb, _, (K, N)), (wqc, wsc) in zip(host, wq):
+        xq, sx = fl.fp8_quant_rows(xb[:rows])
+        fl.fp8_linear(xq, sx, wqc, wsc)
+        flops += 2.0 * rows * N * K
+    return flops, time.perf_counter() - t0
+
+
+def run_fp8_linear(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import action_diffusion_transformers_b200 as adt
+
+    w = synth.WORKLOADS[args.workload]
+    M = w.B * w.N
+    host = []
+    for i, (name, K, N) in enumerate(fp8_shapes(w)):
+        xb, wb = fp8_inputs(w, K, N, w.seed * 10 + i)
+        host.append((xb, wb, (K, N)))
+    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
+    dev = []
+    for xb, wb, (K, N) in host:
+        x = as_dev(xb)
+        wd = as_dev(wb)
+        wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+        sw = torch.empty(N, dtype=torch.float32, device="cuda")
+        adt.sage_fp8_quant_rows(wd, wq, sw)           # offline: the weights' E4M3 codes and row scales
+        del wd
+        xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+        sx = torch.empty(M, dtype=torch.float32, device="cuda")
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        dev.append(dict(x=x, wq=wq, sw=sw, xq=xq, sx=sx, out=out, K=K, N=N))
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flops = sum(2.0 * M * d["N"] * d["K"] for d in dev)
+
+    def step(evs=None):
+        for i, d in enumerate(dev):
+            adt.sage_fp8_quant_rows(d["x"], d["xq"], d["sx"], stream)
+            if evs is not None:
+                evs[i].record(stream)
+            adt.sage_fp8_linear(d["xq"], d["sx"], d["wq"], d["sw"], d["out"], stream)
+            if evs is not None:
+                evs[len(dev) + i].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    adt.sage_check()
+    torch.cuda.synchronize()
+    barrier()
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * len(dev) + 1)] for _ in range(K_steps)]
+    sampler = ClockSampler(gpu_id_for(local))
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(K_steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step(ev[i][1:])
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    adt.sage_check()
+    nd = len(dev)
+    step_ms = [e[0].elapsed_time(e[2 * nd]) for e in ev]
+    max_total_ms = max_over_ranks(sum(step_ms), world, "cuda")
+    value = job_tops(world, flops, K_steps, max_total_ms)
+    quant_us, gemm_us = {}, {}
+    for j, (name, _, _) in enumerate(fp8_shapes(w)):
+        prev = [e[0] if j == 0 else e[nd + j] for e in ev]
+        quant_us[name] = 1e3 * statistics.mean(p.elapsed_time(e[1 + j]) for p, e in zip(prev, ev))
+        gemm_us[name] = 1e3 * statistics.mean(e[1 + j].elapsed_time(e[1 + nd + j]) for e in ev)
+
+    # e2e: pinned host activations in, BF16 projection outputs back, every step
+    hx = [torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory() for xb, _, _ in host]
+    hout = [torch.empty(d["out"].shape, dtype=torch.bfloat16).pin_memory() for d in dev]
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
+
+    def e2e_step():
+        for d, h in zip(dev, hx):
+            d["x"].copy_(h, non_blocking=True)
+        step()
+        for d, h in zip(dev, hout):
+            h.copy_(d["out"], non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    for i in range(K_steps):
+        flush.fill_(i & 0xFF)
+        e2e_ev[i][0].record(stream)
+        e2e_step()
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    adt.sage_check()
+    e2e_value = job_tops(world, flops, K_steps, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world,
+                                                                "cuda"))
+    h2d = sum(xb.nbytes for xb, _, _ in host)
+    d2h = sum(d["out"].numel() * 2 for d in dev)
+
+    peaks, src = load_peaks()
+    peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    # the dominant launch: the MLP up-projection
+    _, k_up, n_up = fp8_shapes(w)[1]
+    achieved = 2.0 * M * n_up * k_up / (gemm_us["mlp_up"] / 1e6) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = 16
+        o_flops, o_dt = fp8_oracle_sample(w, host, rows)
+        cpu = {"value": o_flops / o_dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{rows} tokens through each of the {len(dev)} projections ({o_dt:.1f} s)"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    x_bytes = sum(M * d["K"] * (2 + 1) + M * 4 for d in dev)
+    line = {
+        "metric": "fp8 projection TFLOPS", "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": max_total_ms / K_steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": f"{w.name} joint-block projections", "tokens": M, "hidden": w.H * w.D,
+                   "shapes": {n: [M, N, K] for n, K, N in fp8_shapes(w)}, "global_batch": w.B * world,
+                   "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "traffic": kernel_traffic("fp8_gemm_kernel", ("fp8_linear.cuh", "sage_ptx.cuh"),
+                                               f"{w.name} mlp_up"),
+                     "kernel": "fp8_gemm_kernel (mlp_up launch)",
+                     "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (fp8 dense)"},
+        "kernels_us": {"quant_x": quant_us, "gemm": gemm_us},
+        "quant_gbs": x_bytes / (sum(quant_us.values()) / 1e6) / 1e9,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * len(dev) * K_steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- ours
 def main():
     args = parse()
@@ -294,6 +517,9 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    if args.op == "fp8_linear":
+        run_fp8_linear(args, rank, world, local)
+        return
     w = synth.WORKLOADS[args.workload]
     qb, kb, vb = synth.generate(w)
     nr_host = None
