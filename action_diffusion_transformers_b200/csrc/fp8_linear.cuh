@@ -6,10 +6,11 @@
 //  fp8_quant_rows_kernel  one CTA per row: absmax, scale = RN(amax/448),
 //                         inv = RN(448/amax), codes = E4M3(RN(x * inv)).
 //  fp8_gemm_kernel        persistent, one CTA per SM over 128 x 256 output
-//                         tiles.  Warp 0 issues TMA loads of 128 x 128 A and
-//                         256 x 128 B tiles into a 4-stage ring; warp 1
-//                         issues tcgen05.mma kind::f8f6f4 (M 128, N 256, K 32)
-//                         into one of two 256-column TMEM accumulators; warps
+//                         (or 128 x 192) tiles.  Warp 0 issues TMA loads of
+//                         128 x 128 A and BN x 128 B tiles into a 4- or 5-stage
+//                         ring; warp 1 issues tcgen05.mma kind::f8f6f4 (M 128,
+//                         N BN, K 32) into one of two BN-column TMEM
+//                         accumulators; warps
 //                         2-5 (one per TMEM lane quadrant) read the other
 //                         accumulator, apply the two scales and store BF16 or
 //                         FP32, so a tile's epilogue overlaps the next tile's
@@ -80,21 +81,24 @@ __global__ void __launch_bounds__(kFqThreads) fp8_quant_rows_kernel(const uint16
 // Persistent FP8 GEMM with row-wise scales.
 // ----------------------------------------------------------------------------
 constexpr int kGemmBM = 128;        // rows of X per tile (TMEM lanes)
-constexpr int kGemmBN = 256;        // rows of W per tile (TMEM columns per accumulator)
 constexpr int kGemmBK = 128;        // K bytes (= E4M3 elements) per stage: one 128 B swizzle row
-constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
+// BN rows of W per tile (TMEM columns per accumulator): 256, or 192 where it
+// fills the last wave of the persistent grid better.  Stages: as many 16 KB +
+// BN * 128 B ring slots as fit next to the barriers.
+template <int BN>
 struct GemmSmem {
+  static constexpr int kStages = BN == 256 ? 4 : 5;
   static constexpr int kABytes = kGemmBM * kGemmBK;
-  static constexpr int kBBytes = kGemmBN * kGemmBK;
+  static constexpr int kBBytes = BN * kGemmBK;
   static constexpr int kA = 0;
-  static constexpr int kB = kA + kGemmStages * kABytes;
-  static constexpr int kBar = kB + kGemmStages * kBBytes;
+  static constexpr int kB = kA + kStages * kABytes;
+  static constexpr int kBar = kB + kStages * kBBytes;
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
-  static constexpr int kFull = 0, kEmpty = kGemmStages, kAccFull = 2 * kGemmStages,
-                       kAccEmpty = 2 * kGemmStages + 2, kDrain = 2 * kGemmStages + 4;
-  static constexpr int kNumBars = 2 * kGemmStages + 5;
+  static constexpr int kFull = 0, kEmpty = kStages, kAccFull = 2 * kStages, kAccEmpty = 2 * kStages + 2,
+                       kDrain = 2 * kStages + 4;
+  static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kMisc = kBar + kNumBars * 8;   // tmem slot, abort flag
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;        // slack for 1024-byte alignment
@@ -110,10 +114,14 @@ struct GemmParams {
   int64_t timeout_ns;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const GemmParams prm) {
-  using L = GemmSmem;
+  using L = GemmSmem<BN>;
+  constexpr int kGemmBN = BN;
+  constexpr int kGemmStages = L::kStages;
+  constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256u : 512u;   // power of two
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
@@ -129,7 +137,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int64_t tmo = prm.timeout_ns;
 
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * kGemmBN);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -273,7 +281,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (*abort_flag && tid == 0) atomicExch(prm.err, 1);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * kGemmBN);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
