@@ -3,8 +3,8 @@
 TEST INFRASTRUCTURE ONLY (part of the CPU oracle; it writes no stored value).
 
 2^f on f in [-1/2, 1/2] is approximated by p(f) = 1 + c1 f + ... + c_d f^d with
-c0 fixed at 1 (so that 2^n is exact at integers): a cubic (d = 3) for the
-per-key weights and a quintic (d = 5) for the once-per-tile rescale factor.
+c0 fixed at 1 (so that 2^n is exact at integers): a quadratic (d = 2) for
+the per-key weights and a quintic (d = 5) for the once-per-tile rescale factor.
 c1..c_d minimise the maximum
 relative error |p(f) / 2^f - 1| on a dense grid, as a linear program
 (minimise t subject to -t <= p(f_i) / 2^f_i - 1 <= t), and are then rounded to
@@ -19,7 +19,7 @@ from __future__ import annotations
 import numpy as np
 from scipy.optimize import linprog
 
-DEGREES = (3, 5)
+DEGREES = (2, 5)
 
 
 def fit(degree: int, points: int = 4001) -> np.ndarray:

@@ -222,14 +222,14 @@ def test_closed_form_dominant_key():
     # The other keys keep the exact softmax weight 1 - w200 of the dequantized
     # scores (E4M3 rounding of their P moves it by < 10%); and key 200's code is
     # E4M3(y) = 448 while the row sum holds y itself, whose exp2 is within the
-    # cubic's 1.013e-4, so the centred output moves by up to that ratio.
+    # quadratic's 1.963e-3, so the centred output moves by up to that ratio.
     qd = it["q_codes"][0, 0, 5].astype(np.float64) * it["q_scale"][0, 0, 0]
     kd = it["k_codes"][0, 0, :N].astype(np.float64) * np.repeat(it["k_scale"][0, 0], 64)[:N, None]
     s = kd @ qd / 8.0
     w = np.exp(s - s.max())
     w /= w.sum()
     spread = np.abs(dec_all - dec).max(axis=0)
-    tol = 1.1 * (1 - w[200]) * spread + 1.02e-4 * np.abs(dec - it["v_mean"][0, 0]) + 1e-6
+    tol = 1.1 * (1 - w[200]) * spread + 1.97e-3 * np.abs(dec - it["v_mean"][0, 0]) + 1e-6
     assert w[200] > 0.999
     assert np.all(np.abs(o[0, 5, 0] - dec) <= tol)
 
@@ -270,9 +270,9 @@ def test_lse_matches_dequantized_logsumexp():
     kd = it["k_codes"][0, 0, :N].astype(np.float64) * np.repeat(it["k_scale"][0, 0], 64)[:N, None]
     s = (qd @ kd.T) / 8.0
     ref = np.log(np.exp(s - s.max(1, keepdims=True)).sum(1)) + s.max(1)
-    # l sums weights with relative error <= 1.013e-4 (the cubic's bound); the
+    # l sums weights with relative error <= 1.963e-3 (the quadratic's bound); the
     # rescale factors use the quintic (2.2e-7)
-    assert np.abs(lse[0, 0] - ref).max() <= 1.03e-4
+    assert np.abs(lse[0, 0] - ref).max() <= 1.97e-3
 
 
 def test_two_pass_variant_close_to_online():
@@ -302,19 +302,19 @@ def test_running_max_with_large_logit_gap():
     dec = nm.e4m3_decode(it["v_codes_t"][0, 0, :, 10]) * it["v_scale"][0, 0] + it["v_mean"][0, 0]
     # The dominant key's exponent is S*c - RN(S*c) + (RN(log2 448 - m) - (log2 448 - m)):
     # off by at most one FP32 ulp of the row max m (here ~1150), and its exp2 is
-    # within the cubic's 1.013e-4, while its code is 448 either way: the centred
-    # output moves by up to ln2 * ulp(m) + 1.013e-4 relative.
+    # within the quadratic's 1.963e-3, while its code is 448 either way: the centred
+    # output moves by up to ln2 * ulp(m) + 1.963e-3 relative.
     S = it["q_codes"][0, 0, 5].astype(np.float64) @ it["k_codes"][0, 0, 10].astype(np.float64)
     c = nm.rn32(nm.rn32(np.float64(it["q_scale"][0, 0, 0]) * it["k_scale"][0, 0, 0])
                 * np.float64(so.exp2_scale(so.default_sm_scale(D))))
     m = nm.rn32(S * np.float64(c))
     assert m > 512
     centred = np.abs(dec - it["v_mean"][0, 0])                  # the part scaled by P8 / l
-    tol = (2 * np.spacing(np.float32(m)) + 1.02e-4) * centred + 1e-6
+    tol = (2 * np.spacing(np.float32(m)) + 1.97e-3) * centred + 1e-6
     assert np.all(np.abs(o[0, 5, 0] - dec) <= tol)
 
 
-@pytest.mark.parametrize("coeffs,bound", [(so.EXP2_C, 1.02e-4), (so.EXP2_C5, 2.3e-7)])
+@pytest.mark.parametrize("coeffs,bound", [(so.EXP2_C, 1.97e-3), (so.EXP2_C5, 2.3e-7)])
 def test_exp2_contract_error_bound_and_exact_points(coeffs, bound):
     rng = np.random.default_rng(21)
     u = np.concatenate([rng.uniform(-125, 9.5, 200000), np.arange(-125, 10) + 0.5,
@@ -332,5 +332,5 @@ def test_exp2_contract_error_bound_and_exact_points(coeffs, bound):
 
 def test_exp2_contract_coefficients_come_from_the_fit():
     fit_exp2 = pytest.importorskip("oracle.fit_exp2")
-    for degree, coeffs in ((3, so.EXP2_C), (5, so.EXP2_C5)):
+    for degree, coeffs in ((2, so.EXP2_C), (5, so.EXP2_C5)):
         assert np.allclose(fit_exp2.fit(degree), np.asarray(coeffs, np.float32), rtol=2e-6, atol=0)
