@@ -133,9 +133,7 @@ __device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const C
 #pragma unroll
     for (int i = 0; i < 8; ++i) f[i] = x2_sub(u[i], f[i]);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) p[i] = x2_fma(k.c3, f[i], k.c2);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c1);
+    for (int i = 0; i < 8; ++i) p[i] = x2_fma(k.c2, f[i], k.c1);
 #pragma unroll
     for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c0);
 #pragma unroll
