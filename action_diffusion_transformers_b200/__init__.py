@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
                 4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_DEVICE_TIMEOUT", 6: "SAGE_ERR_WORKSPACE"}
 EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
             "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error",
-            "sage_quant_qk_static", "sage_quant_qk_normrope", "sage_fp8_quant_rows", "sage_fp8_linear")
+            "sage_quant_qk_static", "sage_quant_qk_normrope", "sage_fp8_quant_rows", "sage_fp8_linear",
+            "sage_quant_qkv")
 QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -62,6 +63,9 @@ _lib.sage_quant_qk_static.restype = ctypes.c_int
 _lib.sage_quant_qk_normrope.argtypes = [_vp, _vp, SageShape, ctypes.POINTER(SageNormRope), _vp, _vp, _vp, _vp, _vp,
                                         _vp, ctypes.c_size_t, _vp]
 _lib.sage_quant_qk_normrope.restype = ctypes.c_int
+_lib.sage_quant_qkv.argtypes = [_vp, _vp, _vp, SageShape, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp, ctypes.c_size_t, _vp]
+_lib.sage_quant_qkv.restype = ctypes.c_int
 _lib.sage_fp8_quant_rows.argtypes = [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int64, _vp, _vp, _vp]
 _lib.sage_fp8_quant_rows.restype = ctypes.c_int
 _lib.sage_fp8_linear.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp, ctypes.c_int,
@@ -162,6 +166,16 @@ def sage_quant_qk_normrope(q, k, shape, q_weight, k_weight, rope_cos, rope_sin, 
         "sage_quant_qk_normrope")
 
 
+def sage_quant_qkv(q, k, v, shape, v_tok_stride, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes_t, v_scale,
+                   v_mean, workspace, stream=None):
+    """sage_quant_qk and sage_quant_v in three launches (identical outputs); v may
+    have its own token stride (0 means H*D)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
+    _ok(_lib.sage_quant_qkv(_ptr(q), _ptr(k), _ptr(v), shape, int(v_tok_stride), _ptr(q_codes), _ptr(q_scale),
+                            _ptr(k_codes), _ptr(k_scale), _ptr(k_mean), _ptr(v_codes_t), _ptr(v_scale), _ptr(v_mean),
+                            _ptr(workspace), ws_bytes, _stream(stream)), "sage_quant_qkv")
+
+
 def sage_fp8_quant_rows(x, codes, scale, stream=None):
     """Per-row E4M3 codes [R, K] (uint8) and scales [R] (float32) of a BF16 [R, K]
     tensor whose rows may be strided (x.stride(1) must be 1)."""
@@ -237,14 +251,16 @@ class Buffers:
         None, or dict(q_w, k_w, cos, sin, eps) of device tensors (and a float): Q and K
         are then projection outputs, normed and rotated inside the quantization."""
         if normrope is None:
-            sage_quant_qk(q, k, self.shape, self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.k_mean,
-                          self.workspace, stream)
+            sage_quant_qkv(q, k, v, self.shape, (v_shape or self.shape).tok_stride, self.q_codes, self.q_scale,
+                           self.k_codes, self.k_scale, self.k_mean, self.v_codes_t, self.v_scale, self.v_mean,
+                           self.workspace, stream)
         else:
             nr = normrope
             sage_quant_qk_normrope(q, k, self.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
                                    self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.k_mean,
                                    self.workspace, stream)
-        sage_quant_v(v, v_shape or self.shape, self.v_codes_t, self.v_scale, self.v_mean, self.workspace, stream)
+            sage_quant_v(v, v_shape or self.shape, self.v_codes_t, self.v_scale, self.v_mean, self.workspace,
+                         stream)
         sage_attn_fwd(self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.v_codes_t, self.v_scale,
                       self.v_mean, self.shape, sm_scale, self.out, self.out_fp32, self.lse, stream)
         return self.out

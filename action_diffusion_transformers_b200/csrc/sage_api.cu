@@ -162,7 +162,7 @@ sage_status check_shape(const sage_shape& s, int64_t* tok_stride) {
 }
 
 struct WsLayout {
-  size_t psum, pmin, pmax, kmean, vinv, total;
+  size_t psum, pmin, pmax, kmean, vinv, psum_v, single, total;
 };
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 WsLayout ws_layout(const sage_shape& s) {
@@ -175,16 +175,19 @@ WsLayout ws_layout(const sage_shape& s) {
   w.pmax = align256(w.pmin + part * 4);
   w.kmean = align256(w.pmax + part * 4);
   w.vinv = align256(w.kmean + chans * 2);
-  w.total = align256(w.vinv + chans * 4);
+  w.single = align256(w.vinv + chans * 4);      // what sage_quant_qk or sage_quant_v alone needs
+  w.psum_v = w.single;                          // sage_quant_qkv: V partials beside K's
+  w.total = align256(w.psum_v + part * 8);
   return w;
 }
 
-sage_status check_ws(const sage_shape& s, const void* ws, size_t ws_bytes, WsLayout* lay) {
+sage_status check_ws(const sage_shape& s, const void* ws, size_t ws_bytes, WsLayout* lay, bool fused = false) {
   *lay = ws_layout(s);
+  const size_t need = fused ? lay->total : lay->single;
   if (!ws) return fail(SAGE_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(SAGE_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
-  if (ws_bytes < lay->total)
-    return fail(SAGE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, lay->total);
+  if (ws_bytes < need)
+    return fail(SAGE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
   return SAGE_OK;
 }
 
@@ -383,6 +386,74 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
                                                                 static_cast<uint16_t*>(k_mean));
   launch_qk_codes<false>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, sage::NormRopeArgs{}, cs);
   return launch_check("sage_quant_qk launch");
+}
+
+sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_shape s, int64_t v_tok_stride,
+                           int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale, void* k_mean,
+                           uint8_t* v_codes_t, float* v_scale, float* v_mean, void* workspace, size_t ws_bytes,
+                           sage_stream_t stream) {
+  if (s.q_gran != SAGE_GRAN_BLOCK64 || s.k_gran != SAGE_GRAN_BLOCK64) {
+    // finer scale groups: the two calls one after the other
+    sage_status st = sage_quant_qk(q, k, s, q_codes, q_scale, k_codes, k_scale, k_mean, workspace, ws_bytes,
+                                   stream);
+    if (st != SAGE_OK) return st;
+    sage_shape sv = s;
+    sv.tok_stride = v_tok_stride;
+    return sage_quant_v(v, sv, v_codes_t, v_scale, v_mean, workspace, ws_bytes, stream);
+  }
+  int64_t ts, vts;
+  sage_status st = check_shape(s, &ts);
+  if (st != SAGE_OK) return st;
+  sage_shape sv = s;
+  sv.tok_stride = v_tok_stride;
+  if ((st = check_shape(sv, &vts)) != SAGE_OK) return st;
+  if (3LL * s.B > 65535) return fail(SAGE_ERR_INVALID_ARG, "B = %d too large for sage_quant_qkv", s.B);
+  SAGE_NEED(q, "q");
+  SAGE_NEED(k, "k");
+  SAGE_NEED(v, "v");
+  SAGE_NEED(q_codes, "q_codes");
+  SAGE_NEED(q_scale, "q_scale");
+  SAGE_NEED(k_codes, "k_codes");
+  SAGE_NEED(k_scale, "k_scale");
+  SAGE_NEED(v_codes_t, "v_codes_t");
+  SAGE_NEED(v_scale, "v_scale");
+  SAGE_NEED(v_mean, "v_mean");
+  if (k_mean && !aligned16(k_mean)) return fail(SAGE_ERR_ALIGNMENT, "k_mean is not 16-byte aligned");
+  WsLayout lay;
+  if ((st = check_ws(s, workspace, ws_bytes, &lay, true)) != SAGE_OK) return st;
+  int dev;
+  int* err;
+  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  double* psum_k = reinterpret_cast<double*>(ws + lay.psum);
+  double* psum_v = reinterpret_cast<double*>(ws + lay.psum_v);
+  float* pmin = reinterpret_cast<float*>(ws + lay.pmin);
+  float* pmax = reinterpret_cast<float*>(ws + lay.pmax);
+  uint16_t* kmean = reinterpret_cast<uint16_t*>(ws + lay.kmean);
+  float* vinv = reinterpret_cast<float*>(ws + lay.vinv);
+  const int HD = s.H * s.D;
+  const int nsb = (s.N + sage::kSumBlock - 1) / sage::kSumBlock;
+  const int Npad = static_cast<int>(npad_of(s.N));
+  const int zc = (HD + 1023) / 1024;
+  const uint16_t* qb = static_cast<const uint16_t*>(q);
+  const uint16_t* kb = static_cast<const uint16_t*>(k);
+  const uint16_t* vb = static_cast<const uint16_t*>(v);
+
+  sage::colstats_kv<<<dim3(nsb, s.B, 2 * zc), 128, 0, cs>>>(kb, vb, s.N, HD, ts, vts, nsb, zc, psum_k, psum_v, pmin,
+                                                             pmax);
+  const int nf = (s.B * HD + 31) / 32;
+  sage::finalize_kv<<<2 * nf, 1024, 0, cs>>>(psum_k, psum_v, pmin, pmax, s.B, s.N, HD, nsb, nf, kmean,
+                                              static_cast<uint16_t*>(k_mean), v_mean, v_scale, vinv);
+  const dim3 g(Npad / sage::kTile, s.H, 3 * s.B);
+  if (s.D == 128)
+    sage::codes_qkv<128><<<g, 256, 0, cs>>>(qb, kb, vb, s.N, s.B, s.H, Npad, ts, vts, kmean, q_codes, q_scale,
+                                            k_codes, k_scale, v_mean, vinv, v_codes_t);
+  else
+    sage::codes_qkv<64><<<g, 256, 0, cs>>>(qb, kb, vb, s.N, s.B, s.H, Npad, ts, vts, kmean, q_codes, q_scale,
+                                           k_codes, k_scale, v_mean, vinv, v_codes_t);
+  return launch_check("sage_quant_qkv launch");
 }
 
 sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s, const sage_normrope* nr,

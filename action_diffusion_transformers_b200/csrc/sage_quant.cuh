@@ -150,13 +150,12 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
 // token order, in FP64.  Grid (nsb, B, ceil(HD / (8*blockDim))).
 // ----------------------------------------------------------------------------
 template <bool kMinMax>
-__global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restrict__ x, int N, int HD,
-                                                        int64_t tok_stride, int nsb,
-                                                        double* __restrict__ psum,
-                                                        float* __restrict__ pmin, float* __restrict__ pmax) {
-  const int c = blockIdx.x;
-  const int b = blockIdx.y;
-  const int ch0 = (blockIdx.z * blockDim.x + threadIdx.x) * 8;
+__device__ __forceinline__ void colstats_body(int bx, int by, int bz, const uint16_t* __restrict__ x, int N,
+                                              int HD, int64_t tok_stride, int nsb, double* __restrict__ psum,
+                                              float* __restrict__ pmin, float* __restrict__ pmax) {
+  const int c = bx;
+  const int b = by;
+  const int ch0 = (bz * 128 + threadIdx.x) * 8;
   if (ch0 >= HD) return;
   const int n0 = c * kSumBlock;
   const int n1 = min(N, n0 + kSumBlock);
@@ -207,6 +206,14 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
     px[0] = make_float4(__low2float(mx[0]), __high2float(mx[0]), __low2float(mx[1]), __high2float(mx[1]));
     px[1] = make_float4(__low2float(mx[2]), __high2float(mx[2]), __low2float(mx[3]), __high2float(mx[3]));
   }
+}
+
+template <bool kMinMax>
+__global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restrict__ x, int N, int HD,
+                                                        int64_t tok_stride, int nsb,
+                                                        double* __restrict__ psum,
+                                                        float* __restrict__ pmin, float* __restrict__ pmax) {
+  colstats_body<kMinMax>(blockIdx.x, blockIdx.y, blockIdx.z, x, N, HD, tok_stride, nsb, psum, pmin, pmax);
 }
 
 // K column sums (as colstats_partial<false>: same grid, order and output) of
@@ -318,11 +325,10 @@ __device__ __forceinline__ void finalize_channel(const double* __restrict__ psum
   }
 }
 
-__global__ void __launch_bounds__(1024) k_mean_finalize(const double* __restrict__ psum, int B, int N, int HD,
-                                                        int nsb, uint16_t* __restrict__ mean_ws,
-                                                        uint16_t* __restrict__ mean_out) {
-  __shared__ double sh[kSumLanes][33];
-  const int gch = blockIdx.x * 32 + (threadIdx.x & 31);
+__device__ __forceinline__ void k_mean_body(int bx, const double* __restrict__ psum, int B, int N, int HD, int nsb,
+                                            uint16_t* __restrict__ mean_ws, uint16_t* __restrict__ mean_out,
+                                            double (&sh)[kSumLanes][33]) {
+  const int gch = bx * 32 + (threadIdx.x & 31);
   const bool valid = gch < B * HD;
   const int b = valid ? gch / HD : 0;
   const int ch = valid ? gch % HD : 0;
@@ -337,17 +343,21 @@ __global__ void __launch_bounds__(1024) k_mean_finalize(const double* __restrict
   }
 }
 
+__global__ void __launch_bounds__(1024) k_mean_finalize(const double* __restrict__ psum, int B, int N, int HD,
+                                                        int nsb, uint16_t* __restrict__ mean_ws,
+                                                        uint16_t* __restrict__ mean_out) {
+  __shared__ double sh[kSumLanes][33];
+  k_mean_body(blockIdx.x, psum, B, N, HD, nsb, mean_ws, mean_out, sh);
+}
+
 // V: mean = RN_f32(sum / N); amax = max(RN(vmax - mean), RN(mean - vmin));
 // scale = RN(amax / 448), inv = RN(448 / amax) (0, 0 for amax == 0).
-__global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restrict__ psum,
-                                                         const float* __restrict__ pmin,
-                                                         const float* __restrict__ pmax, int B, int N, int HD,
-                                                         int nsb, float* __restrict__ v_mean,
-                                                         float* __restrict__ v_scale, float* __restrict__ v_inv) {
-  __shared__ double sh[kSumLanes][33];
-  __shared__ float shn[kSumLanes][33];
-  __shared__ float shx[kSumLanes][33];
-  const int gch = blockIdx.x * 32 + (threadIdx.x & 31);
+__device__ __forceinline__ void v_stats_body(int bx, const double* __restrict__ psum, const float* __restrict__ pmin,
+                                             const float* __restrict__ pmax, int B, int N, int HD, int nsb,
+                                             float* __restrict__ v_mean, float* __restrict__ v_scale,
+                                             float* __restrict__ v_inv, double (&sh)[kSumLanes][33],
+                                             float (&shn)[kSumLanes][33], float (&shx)[kSumLanes][33]) {
+  const int gch = bx * 32 + (threadIdx.x & 31);
   const bool valid = gch < B * HD;
   const int b = valid ? gch / HD : 0;
   const int ch = valid ? gch % HD : 0;
@@ -368,6 +378,17 @@ __global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restric
   }
 }
 
+__global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restrict__ psum,
+                                                         const float* __restrict__ pmin,
+                                                         const float* __restrict__ pmax, int B, int N, int HD,
+                                                         int nsb, float* __restrict__ v_mean,
+                                                         float* __restrict__ v_scale, float* __restrict__ v_inv) {
+  __shared__ double sh[kSumLanes][33];
+  __shared__ float shn[kSumLanes][33];
+  __shared__ float shx[kSumLanes][33];
+  v_stats_body(blockIdx.x, psum, pmin, pmax, B, N, HD, nsb, v_mean, v_scale, v_inv, sh, shn, shx);
+}
+
 // ----------------------------------------------------------------------------
 // INT8 block quantization.  CTA = one (b, h, 128-token tile = two 64-token
 // scale blocks) of K (z < B: centred by mean_k and rounded to BF16 first) or Q
@@ -385,14 +406,13 @@ __device__ __forceinline__ int rne_small(float y) {
 // kNR: Q and K rows first go through QK RMSNorm + RoPE (norm_rope_rows); that
 // variant takes one 64-token block per CTA (4 rows per thread), so that two
 // CTAs fit an SM and one's loads overlap the other's reduction and stores.
-template <int D, bool kNR = false>
-__global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_t* __restrict__ q,
-                                                      const uint16_t* __restrict__ k, int N, int B, int H,
-                                                      int Npad, int64_t tok_stride,
-                                                      const uint16_t* __restrict__ k_mean,
-                                                      int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
-                                                      int8_t* __restrict__ k_codes,
-                                                      float* __restrict__ k_scale, const NormRopeArgs nr = {}) {
+template <int D, bool kNR>
+__device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint16_t* __restrict__ q,
+                                              const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
+                                              int64_t tok_stride, const uint16_t* __restrict__ k_mean,
+                                              int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+                                              int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
+                                              const NormRopeArgs& nr) {
   constexpr int kWarps = 256 / 32;
   constexpr int kSlots = kNR ? 1 : 2;     // 64-token blocks per CTA
   constexpr int kTokens = kSlots * kQKBlock;
@@ -401,12 +421,12 @@ __global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_
   constexpr int kTPT = kTokens / kRPP;    // tokens per thread (kHalf in each block)
   constexpr int kHalf = kTPT / kSlots;
   __shared__ float red[kWarps][2];
-  const int tile = blockIdx.x;
-  const bool is_k = static_cast<int>(blockIdx.z) < B;
+  const int tile = bx;
+  const bool is_k = static_cast<int>(bz) < B;
   // K heads are visited last-to-first: the column-sum pass just streamed K in
   // head order, so the most recently read heads (still in L2) come first.
-  const int h = is_k ? H - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
-  const int b = is_k ? blockIdx.z : blockIdx.z - B;
+  const int h = is_k ? H - 1 - static_cast<int>(by) : static_cast<int>(by);
+  const int b = is_k ? bz : bz - B;
   const uint16_t* src = is_k ? k : q;
   const int cg = threadIdx.x % kLPR;
   const int r0 = threadIdx.x / kLPR;
@@ -496,6 +516,18 @@ __global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_
   }
   if (threadIdx.x < kSlots)
     (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + tile * kSlots + threadIdx.x] = threadIdx.x == 0 ? scale[0] : scale[1];
+}
+
+template <int D, bool kNR = false>
+__global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_t* __restrict__ q,
+                                                      const uint16_t* __restrict__ k, int N, int B, int H,
+                                                      int Npad, int64_t tok_stride,
+                                                      const uint16_t* __restrict__ k_mean,
+                                                      int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+                                                      int8_t* __restrict__ k_codes,
+                                                      float* __restrict__ k_scale, const NormRopeArgs nr = {}) {
+  qk_block_body<D, kNR>(blockIdx.x, blockIdx.y, blockIdx.z, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes,
+                        q_scale, k_codes, k_scale, nr);
 }
 
 // ----------------------------------------------------------------------------
@@ -731,18 +763,18 @@ __global__ void __launch_bounds__(256, kNR ? 1 : ((kGranQ == kGranSegment64 || k
 // piece of the transposed output row.  Grid (Npad/128, H, B).
 // ----------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v, int N, int H, int Npad,
-                                                 int64_t tok_stride, const float* __restrict__ v_mean,
-                                                 const float* __restrict__ v_inv, uint8_t* __restrict__ out) {
+__device__ __forceinline__ void v_quant_body(int bx, int by, int bz, const uint16_t* __restrict__ v, int N, int H,
+                                             int Npad, int64_t tok_stride, const float* __restrict__ v_mean,
+                                             const float* __restrict__ v_inv, uint8_t* __restrict__ out) {
   constexpr int kLPR = D / 8;
   constexpr int kRPP = 256 / kLPR;
   constexpr int kTPT = kTile / kRPP;
   constexpr int kPitch = D + 16;          // bytes per token row of the shared tile
   __shared__ __align__(16) uint8_t tile[kTile * kPitch];
-  const int n0 = blockIdx.x * kTile;
+  const int n0 = bx * kTile;
   // Heads last-to-first: the statistics pass just streamed V in head order.
-  const int h = H - 1 - static_cast<int>(blockIdx.y);
-  const int b = blockIdx.z;
+  const int h = H - 1 - static_cast<int>(by);
+  const int b = bz;
   const int cg = threadIdx.x % kLPR;
   const int r0 = threadIdx.x / kLPR;
   const int d0 = cg * 8;
@@ -799,6 +831,70 @@ __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v,
       *reinterpret_cast<uint4*>(out + (bhd + 4 * d4 + c) * Npad + n0 + qc * 16) =
           make_uint4(col[c][0], col[c][1], col[c][2], col[c][3]);
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v, int N, int H, int Npad,
+                                                 int64_t tok_stride, const float* __restrict__ v_mean,
+                                                 const float* __restrict__ v_inv, uint8_t* __restrict__ out) {
+  v_quant_body<D>(blockIdx.x, blockIdx.y, blockIdx.z, v, N, H, Npad, tok_stride, v_mean, v_inv, out);
+}
+
+// ----------------------------------------------------------------------------
+// sage_quant_qkv: the passes of sage_quant_qk and sage_quant_v in three
+// launches instead of six (statistics of K and V; both finalizes; Q, K and V
+// codes), so that each launch has enough CTAs to fill the GPU on small
+// shapes.  The CTA bodies are the same functions, so the bytes are identical.
+// ----------------------------------------------------------------------------
+// Grid (nsb, B, zk + zv): z < zk the K column sums (into psum_k), else the V
+// sums, minima and maxima (psum_v, pmin, pmax).
+__global__ void __launch_bounds__(128) colstats_kv(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+                                                   int N, int HD, int64_t k_stride, int64_t v_stride, int nsb,
+                                                   int zk, double* __restrict__ psum_k, double* __restrict__ psum_v,
+                                                   float* __restrict__ pmin, float* __restrict__ pmax) {
+  const int z = static_cast<int>(blockIdx.z);
+  if (z < zk)
+    colstats_body<false>(blockIdx.x, blockIdx.y, z, k, N, HD, k_stride, nsb, psum_k, nullptr, nullptr);
+  else
+    colstats_body<true>(blockIdx.x, blockIdx.y, z - zk, v, N, HD, v_stride, nsb, psum_v, pmin, pmax);
+}
+
+// Grid (nk + nv) of 1024 threads: blocks < nk the K mean, the rest the V
+// statistics (32 channels per block each).
+__global__ void __launch_bounds__(1024) finalize_kv(const double* __restrict__ psum_k,
+                                                    const double* __restrict__ psum_v,
+                                                    const float* __restrict__ pmin, const float* __restrict__ pmax,
+                                                    int B, int N, int HD, int nsb, int nk,
+                                                    uint16_t* __restrict__ mean_ws, uint16_t* __restrict__ mean_out,
+                                                    float* __restrict__ v_mean, float* __restrict__ v_scale,
+                                                    float* __restrict__ v_inv) {
+  __shared__ double sh[kSumLanes][33];
+  __shared__ float shn[kSumLanes][33];
+  __shared__ float shx[kSumLanes][33];
+  const int bx = static_cast<int>(blockIdx.x);
+  if (bx < nk)
+    k_mean_body(bx, psum_k, B, N, HD, nsb, mean_ws, mean_out, sh);
+  else
+    v_stats_body(bx - nk, psum_v, pmin, pmax, B, N, HD, nsb, v_mean, v_scale, v_inv, sh, shn, shx);
+}
+
+// Grid (Npad/128, H, 3B) of 256 threads: z < 2B the Q / K codes of
+// qk_block_quant (K first), the rest the transposed V codes of v_quant_t.
+template <int D>
+__global__ void __launch_bounds__(256, 3) codes_qkv(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                                    const uint16_t* __restrict__ v, int N, int B, int H, int Npad,
+                                                    int64_t qk_stride, int64_t v_stride,
+                                                    const uint16_t* __restrict__ k_mean,
+                                                    int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
+                                                    int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
+                                                    const float* __restrict__ v_mean,
+                                                    const float* __restrict__ v_inv, uint8_t* __restrict__ v_codes) {
+  const int z = static_cast<int>(blockIdx.z);
+  if (z < 2 * B)
+    qk_block_body<D, false>(blockIdx.x, blockIdx.y, z, q, k, N, B, H, Npad, qk_stride, k_mean, q_codes, q_scale,
+                            k_codes, k_scale, NormRopeArgs{});
+  else
+    v_quant_body<D>(blockIdx.x, blockIdx.y, z - 2 * B, v, N, H, Npad, v_stride, v_mean, v_inv, v_codes);
 }
 
 }  // namespace sage

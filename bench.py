@@ -105,6 +105,8 @@ def parse():
                     help="INT8 scale groups of Q (default: 64-token blocks)")
     ap.add_argument("--k-gran", default="block64", choices=["block64", "token", "segment64"],
                     help="INT8 scale groups of K (default: 64-token blocks)")
+    ap.add_argument("--quant", default="fused", choices=["fused", "separate"],
+                    help="fused: sage_quant_qkv (3 launches); separate: sage_quant_qk + sage_quant_v (6)")
     ap.add_argument("--op", default="attention", choices=["attention", "fp8_linear"],
                     help="attention: the quantized attention path (default); fp8_linear: the row-wise "
                          "FP8 projections of a joint block on the same tokens")
@@ -548,6 +550,19 @@ def main():
     def quant_v():
         adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
 
+    fused = args.quant == "fused" and nr is None
+
+    def quant_qkv():
+        adt.sage_quant_qkv(q, k, v, buf.shape, 0, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                           buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
+
+    def quant_all():
+        if fused:
+            quant_qkv()
+        else:
+            quant_qk()
+            quant_v()
+
     def attn():
         adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
                           buf.v_mean, buf.shape, 0.0, buf.out, False, None, stream)
@@ -557,7 +572,7 @@ def main():
             dist.barrier()
 
     for _ in range(max(3, args.warmup)):
-        quant_qk(); quant_v(); attn()
+        quant_all(); attn()
     adt.sage_check()
     torch.cuda.synchronize()
     barrier()
@@ -572,9 +587,12 @@ def main():
         flush.fill_(i & 0xFF)
         e = ev[i]
         e[0].record(stream)
-        quant_qk()
-        e[1].record(stream)
-        quant_v()
+        if fused:
+            quant_qkv()
+        else:
+            quant_qk()
+            e[1].record(stream)
+            quant_v()
         e[2].record(stream)
         attn()
         e[3].record(stream)
@@ -584,8 +602,9 @@ def main():
     adt.sage_check()
 
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    qk_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    v_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    qk_ms = None if fused else [e[0].elapsed_time(e[1]) for e in ev]
+    v_ms = None if fused else [e[1].elapsed_time(e[2]) for e in ev]
     at_ms = [e[2].elapsed_time(e[3]) for e in ev]
     max_total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     ops = w.attn_ops
@@ -598,7 +617,7 @@ def main():
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for _ in range(2):
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        quant_qk(); quant_v(); attn()
+        quant_all(); attn()
         hout.copy_(buf.out, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
@@ -606,7 +625,7 @@ def main():
         flush.fill_(i & 0xFF)
         e2e_ev[i][0].record(stream)
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        quant_qk(); quant_v(); attn()
+        quant_all(); attn()
         hout.copy_(buf.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
@@ -625,6 +644,15 @@ def main():
     qk_bytes, v_bytes = quant_bytes(w, args.q_gran, args.k_gran)
     if nr is not None:
         qk_bytes += w.N * w.D // 2 * 8 + 2 * w.D * 2          # cos / sin tables once, the two weights
+    if fused:
+        quant_us = {"quant_qkv": 1e3 * statistics.mean(quant_ms), "attn": 1e3 * attn_mean_ms}
+        quant_gbs = {"quant_qkv": (qk_bytes + v_bytes) / (statistics.mean(quant_ms) / 1e3) / 1e9,
+                     "peak_hbm_gbs": peaks["hbm_gbs"]}
+    else:
+        quant_us = {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
+                    "attn": 1e3 * attn_mean_ms}
+        quant_gbs = {"quant_qk": qk_bytes / (statistics.mean(qk_ms) / 1e3) / 1e9,
+                     "quant_v": v_bytes / (statistics.mean(v_ms) / 1e3) / 1e9, "peak_hbm_gbs": peaks["hbm_gbs"]}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of CPU work on the GPU machine's host: 4 heads, 2^26 (query row, key) pairs
@@ -651,14 +679,11 @@ def main():
                      "frac": achieved / peak, "traffic": attn_traffic(w.name) if k_blocks else None,
                      "kernel": f"sage_attn_kernel<{w.D}, {'false' if k_blocks else 'true'}>",
                      "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"},
-        "kernels_us": {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
-                       "attn": 1e3 * attn_mean_ms},
-        "quant_gbs": {"quant_qk": qk_bytes / (statistics.mean(qk_ms) / 1e3) / 1e9,
-                      "quant_v": v_bytes / (statistics.mean(v_ms) / 1e3) / 1e9,
-                      "peak_hbm_gbs": peaks["hbm_gbs"]},
+        "kernels_us": quant_us,
+        "quant_gbs": quant_gbs,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 7 * K,
+        "gpu_launches": (4 if fused else 7) * K,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

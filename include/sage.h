@@ -109,8 +109,9 @@ typedef struct {
 /* N rounded up to a whole 128-row tile. */
 SAGE_API size_t sage_npad(int N);
 
-/* Bytes of device workspace needed by sage_quant_qk and sage_quant_v for this
- * shape (one buffer serves both; calls on one stream may share it). */
+/* Bytes of device workspace needed by sage_quant_qk, sage_quant_v and
+ * sage_quant_qkv for this shape (one buffer serves all; calls on one stream
+ * may share it). */
 SAGE_API size_t sage_workspace_bytes(sage_shape s);
 
 /*
@@ -136,6 +137,24 @@ SAGE_API sage_status sage_quant_qk(const void* q, const void* k, sage_shape s,
                           int8_t* q_codes, float* q_scale,
                           int8_t* k_codes, float* k_scale, void* k_mean,
                           void* workspace, size_t ws_bytes, sage_stream_t stream);
+
+/*
+ * sage_quant_qkv - sage_quant_qk and sage_quant_v of one attention call
+ * together: the same outputs, bit for bit, in three kernel launches instead of
+ * six (the K and V statistics, both finalizes, then the Q, K and V codes), so
+ * that each launch has enough blocks to fill the GPU on small shapes.
+ *
+ * in : q, k with s.tok_stride; v with v_tok_stride (0 means H*D).
+ * out: as sage_quant_qk and sage_quant_v.
+ * workspace: >= sage_workspace_bytes(s) bytes (the K and V partial sums are
+ * kept apart here).  With finer scale groups (s.q_gran or s.k_gran not
+ * SAGE_GRAN_BLOCK64) it runs the two calls one after the other.
+ */
+SAGE_API sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_shape s,
+                                    int64_t v_tok_stride, int8_t* q_codes, float* q_scale,
+                                    int8_t* k_codes, float* k_scale, void* k_mean,
+                                    uint8_t* v_codes_t, float* v_scale, float* v_mean,
+                                    void* workspace, size_t ws_bytes, sage_stream_t stream);
 
 /*
  * sage_quant_qk_normrope - sage_quant_qk on Q and K straight from the

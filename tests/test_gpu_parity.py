@@ -164,3 +164,23 @@ def test_wait_timeout_is_reported_and_context_survives(adt):
     assert adt.sage_check_status() == 0        # cleared
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+@pytest.mark.parametrize("B,N,H,D", [(1, 200, 2, 64), (2, 1000, 3, 128), (1, 4096, 24, 128)])
+def test_fused_qkv_quantization_equals_the_two_calls(adt, B, N, H, D):
+    """sage_quant_qkv writes the same bytes as sage_quant_qk + sage_quant_v,
+    with a strided V as well."""
+    w = synth.custom(B, N, H, D, seed=40 + N, k_sigma=4.0, v_sigma=1.0, outlier_frac=0.02)
+    qb, kb, vb = synth.generate(w)
+    wide = np.zeros((B, N, H * D + 64), np.uint16)
+    wide[:, :, 32:32 + H * D] = vb.reshape(B, N, H * D)
+    v_view = _dev(wide)[:, :, 32:32 + H * D]
+    sep = _run_quant(adt, _dev(qb), _dev(kb), v_view, B, N, H, D, v_tok_stride=H * D + 64)
+    fused = adt.Buffers(B, N, H, D, out_fp32=True)
+    adt.sage_quant_qkv(_dev(qb), _dev(kb), v_view, fused.shape, H * D + 64, fused.q_codes, fused.q_scale,
+                       fused.k_codes, fused.k_scale, fused.k_mean, fused.v_codes_t, fused.v_scale, fused.v_mean,
+                       fused.workspace)
+    adt.sage_check()
+    for name in ("q_codes", "q_scale", "k_codes", "k_scale", "k_mean", "v_codes_t", "v_scale", "v_mean"):
+        assert torch.equal(getattr(sep, name), getattr(fused, name)), name
+    _check_quant(fused, so.quant_qk(qb, kb), so.quant_v(vb))
