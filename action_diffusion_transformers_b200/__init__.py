@@ -168,7 +168,7 @@ def sage_quant_qk_normrope(q, k, shape, q_weight, k_weight, rope_cos, rope_sin, 
 
 def sage_quant_qkv(q, k, v, shape, v_tok_stride, q_codes, q_scale, k_codes, k_scale, k_mean, v_codes_t, v_scale,
                    v_mean, workspace, stream=None):
-    """sage_quant_qk and sage_quant_v in three launches (identical outputs); v may
+    """sage_quant_qk and sage_quant_v in four launches (identical outputs); v may
     have its own token stride (0 means H*D)."""
     ws_bytes = workspace.numel() * workspace.element_size() if hasattr(workspace, "numel") else 0
     _ok(_lib.sage_quant_qkv(_ptr(q), _ptr(k), _ptr(v), shape, int(v_tok_stride), _ptr(q_codes), _ptr(q_scale),

@@ -407,7 +407,6 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   sage_shape sv = s;
   sv.tok_stride = v_tok_stride;
   if ((st = check_shape(sv, &vts)) != SAGE_OK) return st;
-  if (3LL * s.B > 65535) return fail(SAGE_ERR_INVALID_ARG, "B = %d too large for sage_quant_qkv", s.B);
   SAGE_NEED(q, "q");
   SAGE_NEED(k, "k");
   SAGE_NEED(v, "v");
@@ -446,13 +445,19 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   const int nf = (s.B * HD + 31) / 32;
   sage::finalize_kv<<<2 * nf, 1024, 0, cs>>>(psum_k, psum_v, pmin, pmax, s.B, s.N, HD, nsb, nf, kmean,
                                               static_cast<uint16_t*>(k_mean), v_mean, v_scale, vinv);
-  const dim3 g(Npad / sage::kTile, s.H, 3 * s.B);
-  if (s.D == 128)
-    sage::codes_qkv<128><<<g, 256, 0, cs>>>(qb, kb, vb, s.N, s.B, s.H, Npad, ts, vts, kmean, q_codes, q_scale,
-                                            k_codes, k_scale, v_mean, vinv, v_codes_t);
-  else
-    sage::codes_qkv<64><<<g, 256, 0, cs>>>(qb, kb, vb, s.N, s.B, s.H, Npad, ts, vts, kmean, q_codes, q_scale,
-                                           k_codes, k_scale, v_mean, vinv, v_codes_t);
+  // The code passes stay two launches: merged, the V blocks would take the Q/K
+  // blocks' register allocation and fit fewer per SM (measured slower).
+  const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
+  const dim3 gv(Npad / sage::kTile, s.H, s.B);
+  if (s.D == 128) {
+    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
+                                                 k_scale);
+    sage::v_quant_t<128><<<gv, 256, 0, cs>>>(vb, s.N, s.H, Npad, vts, v_mean, vinv, v_codes_t);
+  } else {
+    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
+                                                k_scale);
+    sage::v_quant_t<64><<<gv, 256, 0, cs>>>(vb, s.N, s.H, Npad, vts, v_mean, vinv, v_codes_t);
+  }
   return launch_check("sage_quant_qkv launch");
 }
 

@@ -841,10 +841,11 @@ __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v,
 }
 
 // ----------------------------------------------------------------------------
-// sage_quant_qkv: the passes of sage_quant_qk and sage_quant_v in three
-// launches instead of six (statistics of K and V; both finalizes; Q, K and V
-// codes), so that each launch has enough CTAs to fill the GPU on small
-// shapes.  The CTA bodies are the same functions, so the bytes are identical.
+// sage_quant_qkv: the statistics passes of sage_quant_qk and sage_quant_v in
+// one launch and both finalizes in another (the code passes follow as their
+// own two launches), so that each launch has enough CTAs to fill the GPU on
+// small shapes.  The CTA bodies are the same functions, so the bytes are
+// identical.
 // ----------------------------------------------------------------------------
 // Grid (nsb, B, zk + zv): z < zk the K column sums (into psum_k), else the V
 // sums, minima and maxima (psum_v, pmin, pmax).
@@ -876,25 +877,6 @@ __global__ void __launch_bounds__(1024) finalize_kv(const double* __restrict__ p
     k_mean_body(bx, psum_k, B, N, HD, nsb, mean_ws, mean_out, sh);
   else
     v_stats_body(bx - nk, psum_v, pmin, pmax, B, N, HD, nsb, v_mean, v_scale, v_inv, sh, shn, shx);
-}
-
-// Grid (Npad/128, H, 3B) of 256 threads: z < 2B the Q / K codes of
-// qk_block_quant (K first), the rest the transposed V codes of v_quant_t.
-template <int D>
-__global__ void __launch_bounds__(256, 3) codes_qkv(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-                                                    const uint16_t* __restrict__ v, int N, int B, int H, int Npad,
-                                                    int64_t qk_stride, int64_t v_stride,
-                                                    const uint16_t* __restrict__ k_mean,
-                                                    int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
-                                                    int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
-                                                    const float* __restrict__ v_mean,
-                                                    const float* __restrict__ v_inv, uint8_t* __restrict__ v_codes) {
-  const int z = static_cast<int>(blockIdx.z);
-  if (z < 2 * B)
-    qk_block_body<D, false>(blockIdx.x, blockIdx.y, z, q, k, N, B, H, Npad, qk_stride, k_mean, q_codes, q_scale,
-                            k_codes, k_scale, NormRopeArgs{});
-  else
-    v_quant_body<D>(blockIdx.x, blockIdx.y, z - 2 * B, v, N, H, Npad, v_stride, v_mean, v_inv, v_codes);
 }
 
 }  // namespace sage

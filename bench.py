@@ -106,7 +106,7 @@ def parse():
     ap.add_argument("--k-gran", default="block64", choices=["block64", "token", "segment64"],
                     help="INT8 scale groups of K (default: 64-token blocks)")
     ap.add_argument("--quant", default="fused", choices=["fused", "separate"],
-                    help="fused: sage_quant_qkv (3 launches); separate: sage_quant_qk + sage_quant_v (6)")
+                    help="fused: sage_quant_qkv (4 launches); separate: sage_quant_qk + sage_quant_v (6)")
     ap.add_argument("--op", default="attention", choices=["attention", "fp8_linear"],
                     help="attention: the quantized attention path (default); fp8_linear: the row-wise "
                          "FP8 projections of a joint block on the same tokens")
@@ -683,7 +683,7 @@ def main():
         "quant_gbs": quant_gbs,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (4 if fused else 7) * K,
+        "gpu_launches": (5 if fused else 7) * K,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -140,9 +140,10 @@ SAGE_API sage_status sage_quant_qk(const void* q, const void* k, sage_shape s,
 
 /*
  * sage_quant_qkv - sage_quant_qk and sage_quant_v of one attention call
- * together: the same outputs, bit for bit, in three kernel launches instead of
- * six (the K and V statistics, both finalizes, then the Q, K and V codes), so
- * that each launch has enough blocks to fill the GPU on small shapes.
+ * together: the same outputs, bit for bit, in four kernel launches instead of
+ * six (the K and V statistics in one, both finalizes in one, then the Q/K and
+ * the V codes), so that the short statistics passes fill the GPU on small
+ * shapes.
  *
  * in : q, k with s.tok_stride; v with v_tok_stride (0 means H*D).
  * out: as sage_quant_qk and sage_quant_v.
