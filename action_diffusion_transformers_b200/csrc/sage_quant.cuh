@@ -785,6 +785,13 @@ __device__ __forceinline__ void v_quant_body(int bx, int by, int bz, const uint1
     mean[i] = v_mean[bhd + d0 + i];
     inv[i] = v_inv[bhd + d0 + i];
   }
+  uint4 raw[kTPT];                        // every row's load in flight before any is used
+#pragma unroll
+  for (int t = 0; t < kTPT; ++t) {
+    const int n = n0 + r0 + t * kRPP;
+    raw[t] = n < N ? ld_nc_16(v + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
+                   : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
     const int nl = r0 + t * kRPP;
@@ -792,7 +799,7 @@ __device__ __forceinline__ void v_quant_body(int bx, int by, int bz, const uint1
     uint32_t w0 = 0u, w1 = 0u;
     if (n < N) {
       float f[8];
-      unpack8(ld_nc_16(v + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0), f);
+      unpack8(raw[t], f);
       float y[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fsub_rn(f[i], mean[i]), inv[i]);
