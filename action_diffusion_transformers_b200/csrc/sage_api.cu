@@ -99,6 +99,12 @@ sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullpt
         e = cudaFuncSetAttribute(sage::sage_attn_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::AttnSmem<64>::kAlloc);
       if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::v_codes_tma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::VbSmem<128>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::v_codes_tma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::VbSmem<64>::kAlloc);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::GemmSmem<256>::kAlloc);
       if (e == cudaSuccess)
@@ -294,6 +300,28 @@ void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const 
   else with_k(G2{});
 }
 
+// The V code pass of sage_quant_qkv: persistent, TMA staged (v_codes_tma), two
+// CTAs per SM.
+template <int D>
+sage_status launch_v_codes(const sage_shape& s, int Npad, int64_t vts, const uint16_t* vb, const float* v_mean,
+                           const float* vinv, uint8_t* v_codes_t, int* err, int sm_count, cudaStream_t cs) {
+  // V as a [B*N, tok_stride] BF16 matrix; one box = 128 token rows x D channels.
+  CUtensorMap tv;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(vts), static_cast<cuuint64_t>(s.B) * s.N};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(vts) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(sage::kTile)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(vb), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SAGE_ERR_CUDA, "cuTensorMapEncodeTiled (V rows) failed (%d)", static_cast<int>(r));
+  const int total = (Npad / sage::kTile) * s.H * s.B;
+  const int grid = std::min(total, 2 * (sm_count > 0 ? sm_count : 148));
+  sage::v_codes_tma<D><<<grid, sage::kVbThreads, sage::VbSmem<D>::kAlloc, cs>>>(
+      tv, vb, s.N, s.H, s.B, Npad, vts, v_mean, vinv, v_codes_t, err, g_timeout_ns.load());
+  return SAGE_OK;
+}
+
 template <int D>
 __global__ void selftest_wait_kernel(int64_t timeout_ns, int* err) {
   __shared__ uint64_t bar;
@@ -422,7 +450,8 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   if ((st = check_ws(s, workspace, ws_bytes, &lay, true)) != SAGE_OK) return st;
   int dev;
   int* err;
-  if ((st = device_setup(&dev, &err)) != SAGE_OK) return st;
+  int sm_count = 0;
+  if ((st = device_setup(&dev, &err, &sm_count)) != SAGE_OK) return st;
 
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -452,11 +481,13 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   if (s.D == 128) {
     sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
                                                  k_scale);
-    sage::v_quant_t<128><<<gv, 256, 0, cs>>>(vb, s.N, s.H, Npad, vts, v_mean, vinv, v_codes_t);
+    if ((st = launch_v_codes<128>(s, Npad, vts, vb, v_mean, vinv, v_codes_t, err, sm_count, cs)) != SAGE_OK)
+      return st;
   } else {
     sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
                                                 k_scale);
-    sage::v_quant_t<64><<<gv, 256, 0, cs>>>(vb, s.N, s.H, Npad, vts, v_mean, vinv, v_codes_t);
+    if ((st = launch_v_codes<64>(s, Npad, vts, vb, v_mean, vinv, v_codes_t, err, sm_count, cs)) != SAGE_OK)
+      return st;
   }
   return launch_check("sage_quant_qkv launch");
 }

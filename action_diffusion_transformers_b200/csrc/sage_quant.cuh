@@ -848,6 +848,169 @@ __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v,
 }
 
 // ----------------------------------------------------------------------------
+// Persistent V code pass with TMA staging: the same arithmetic and bytes as
+// v_quant_t, but one producer thread copies each 128-token tile (a 2-D TMA box
+// of 128 token rows x D channels of V seen as [B*N, tok_stride], completion
+// counted on an mbarrier) into a 2-stage ring while 8 consumer warps quantize
+// the other stage and write it transposed.  Work items (b, h, 128-token tile)
+// go round robin over the grid (two CTAs per SM).  Every wait is bounded; a
+// timeout raises the error word.
+// ----------------------------------------------------------------------------
+constexpr int kVbStages = 2;
+constexpr int kVbConsumers = 256;
+constexpr int kVbThreads = kVbConsumers + 32;
+
+__device__ __forceinline__ void consumer_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kVbConsumers) : "memory");
+}
+
+template <int D>
+struct VbSmem {
+  static constexpr int kRowBytes = 2 * D;
+  static constexpr int kStageBytes = kTile * kRowBytes;
+  static constexpr int kPitch = D + 16;
+  static constexpr int kTileT = kVbStages * kStageBytes;       // transposed code tile
+  static constexpr int kBar = kTileT + kTile * kPitch;          // full[S], empty[S]
+  static constexpr int kMisc = kBar + 2 * kVbStages * 8;        // abort flag
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 128;                   // slack for 128-byte alignment
+};
+
+template <int D>
+__global__ void __launch_bounds__(kVbThreads, 2)
+    v_codes_tma(const __grid_constant__ CUtensorMap tm_v, const uint16_t* __restrict__ v, int N, int H, int B,
+                 int Npad, int64_t tok_stride, const float* __restrict__ v_mean, const float* __restrict__ v_inv,
+                 uint8_t* __restrict__ out, int* err, int64_t timeout_ns) {
+  using L = VbSmem<D>;
+  constexpr int kLPR = D / 8;
+  constexpr int kRPP = kVbConsumers / kLPR;
+  constexpr int kTPT = kTile / kRPP;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* empty = full + kVbStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
+  uint8_t* tile = smem + L::kTileT;
+  const int ntiles = Npad / kTile;
+  const int total = ntiles * H * B;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < kVbStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kVbConsumers);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (tid >= kVbConsumers) {
+    // ------------------------------------------------------------ producer warp
+    const int lane = tid - kVbConsumers;
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
+      const int s = static_cast<int>(it % kVbStages);
+      const uint32_t use = it / kVbStages;
+      bool ok = true;
+      if (lane == 0 && use > 0) ok = mbar_wait_bounded(&empty[s], (use - 1) & 1, abort_flag, timeout_ns);
+      if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) break;
+      const int tl = item % ntiles;
+      const int h = H - 1 - (item / ntiles) % H;   // heads last-to-first, as v_quant_t
+      const int b = item / (ntiles * H);
+      const int n0 = tl * kTile;
+      // One 2-D copy: rows b*N + n0 .. +127 of V seen as [B*N, tok_stride] BF16, columns
+      // h*D .. +D-1.  Rows past this batch (or past B*N, zero-filled) are never read.
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(L::kStageBytes));
+        tma_load_2d(smem + s * L::kStageBytes, &tm_v, h * D, b * N + n0, &full[s]);
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      // Drain: wait (bounded) for the last copy issued into each ring slot.
+      int no_abort = 0;
+      volatile int* nf = reinterpret_cast<volatile int*>(&no_abort);
+      for (uint32_t s = 0; s < kVbStages; ++s)
+        if (it > s) {
+          const uint32_t last = ((it - 1 - s) / kVbStages) * kVbStages + s;
+          mbar_wait_bounded(&full[s], (last / kVbStages) & 1, nf, 200000000);
+        }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int cg = tid % kLPR;
+    const int r0 = tid / kLPR;
+    const int d0 = cg * 8;
+    uint32_t it = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x, ++it) {
+      const int s = static_cast<int>(it % kVbStages);
+      const int tl = item % ntiles;
+      const int h = H - 1 - (item / ntiles) % H;
+      const int b = item / (ntiles * H);
+      const int n0 = tl * kTile;
+      const int64_t bhd = (static_cast<int64_t>(b) * H + h) * D;
+      float mean[8], inv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        mean[i] = v_mean[bhd + d0 + i];
+        inv[i] = v_inv[bhd + d0 + i];
+      }
+      // Every consumer leaves its bounded wait; a timeout has raised the abort flag,
+      // which all 256 read after the barrier and leave the loop together.
+      mbar_wait_bounded(&full[s], (it / kVbStages) & 1, abort_flag, timeout_ns);
+      consumer_bar_sync();
+      if (*abort_flag) break;
+      const uint8_t* st = smem + s * L::kStageBytes;
+#pragma unroll
+      for (int t = 0; t < kTPT; ++t) {
+        const int nl = r0 + t * kRPP;
+        const int n = n0 + nl;
+        uint32_t w0 = 0u, w1 = 0u;
+        if (n < N) {
+          float f[8];
+          unpack8(*reinterpret_cast<const uint4*>(st + nl * L::kRowBytes + 2 * d0), f);
+          float y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fsub_rn(f[i], mean[i]), inv[i]);
+          w0 = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
+          w1 = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
+        }
+        *reinterpret_cast<uint2*>(tile + nl * L::kPitch + d0) = make_uint2(w0, w1);
+      }
+      mbar_arrive(&empty[s]);              // this stage's rows are consumed
+      consumer_bar_sync();                 // the code tile is complete
+      constexpr int kUnits = (D / 4) * (kTile / 16);
+      for (int u = tid; u < kUnits; u += kVbConsumers) {
+        const int d4 = u % (D / 4);
+        const int qc = u / (D / 4);
+        uint32_t col[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            r[i] = *reinterpret_cast<const uint32_t*>(tile + (qc * 16 + 4 * j + i) * L::kPitch + 4 * d4);
+          const uint32_t lo01 = __byte_perm(r[0], r[1], 0x5140);
+          const uint32_t lo23 = __byte_perm(r[2], r[3], 0x5140);
+          const uint32_t hi01 = __byte_perm(r[0], r[1], 0x7362);
+          const uint32_t hi23 = __byte_perm(r[2], r[3], 0x7362);
+          col[0][j] = __byte_perm(lo01, lo23, 0x5410);
+          col[1][j] = __byte_perm(lo01, lo23, 0x7632);
+          col[2][j] = __byte_perm(hi01, hi23, 0x5410);
+          col[3][j] = __byte_perm(hi01, hi23, 0x7632);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(out + (bhd + 4 * d4 + c) * Npad + n0 + qc * 16) =
+              make_uint4(col[c][0], col[c][1], col[c][2], col[c][3]);
+      }
+      consumer_bar_sync();                 // the code tile is free for the next item
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && tid == 0) atomicExch(err, 1);
+}
+
+// ----------------------------------------------------------------------------
 // sage_quant_qkv: the statistics passes of sage_quant_qk and sage_quant_v in
 // one launch and both finalizes in another (the code passes follow as their
 // own two launches), so that each launch has enough CTAs to fill the GPU on
