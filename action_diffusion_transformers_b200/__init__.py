@@ -246,7 +246,7 @@ class Buffers:
         self.workspace = torch.empty(max(256, workspace_bytes(self.shape)), dtype=torch.uint8, device=dev)
 
     def run(self, q, k, v, sm_scale=0.0, stream=None, v_shape=None, normrope=None):
-        """quant_qk -> quant_v -> attn_fwd; q, k, v are BF16 [B, N, H, D] device tensors
+        """quant_qkv -> attn_fwd; q, k, v are BF16 [B, N, H, D] device tensors
         (v may be a token-strided view; pass v_shape with its tok_stride).  normrope:
         None, or dict(q_w, k_w, cos, sin, eps) of device tensors (and a float): Q and K
         are then projection outputs, normed and rotated inside the quantization."""
