@@ -272,8 +272,10 @@ __global__ void __launch_bounds__(128) colstats_normrope(const uint16_t* __restr
 // blocks g, g+32, g+64, ... in increasing order from +0; then the butterfly
 // u_g <- u_g + u_{g^o} for o = 16, 8, 4, 2, 1; the result is lane 0's value.
 // Block of 1024 threads = 32 lanes (warps) x 32 channels (lanes of a warp, so
-// every load is one coalesced 256-byte row of partials); the channel index
-// runs over B*HD.  For V the same pass also reduces min / max (order-free).
+// every load is one coalesced 256-byte row of partials); one transpose through
+// shared memory then gives warp g channel g's 32 partials, and the butterfly
+// runs on shuffles.  The channel index runs over B*HD.  For V the same pass
+// also reduces min / max (order-free).
 template <bool kMinMax>
 __device__ __forceinline__ void finalize_channel(const double* __restrict__ psum,
                                                  const float* __restrict__ pmin,
@@ -301,27 +303,27 @@ __device__ __forceinline__ void finalize_channel(const double* __restrict__ psum
     shx[g][cl] = mx;
   }
   __syncthreads();
-  // Butterfly across the 32 lanes, every thread computing its own lane g.
+  // Transposed: warp g now holds channel g's 32 lane partials (lane j: lane
+  // j's partial), and the butterfly runs on shuffles; each lane adds its own
+  // value and its partner's in that order, the pairing of the fixed order.
+  double v = sh[cl][g];
+  float vn = 0.f, vx = 0.f;
+  if (kMinMax) {
+    vn = shn[cl][g];
+    vx = shx[cl][g];
+  }
 #pragma unroll
   for (int o = kSumLanes / 2; o >= 1; o >>= 1) {
-    const double w = __dadd_rn(sh[g][cl], sh[g ^ o][cl]);
-    float wn = 0.f, wx = 0.f;
+    v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
     if (kMinMax) {
-      wn = fminf(shn[g][cl], shn[g ^ o][cl]);
-      wx = fmaxf(shx[g][cl], shx[g ^ o][cl]);
+      vn = fminf(vn, __shfl_xor_sync(0xFFFFFFFFu, vn, o));
+      vx = fmaxf(vx, __shfl_xor_sync(0xFFFFFFFFu, vx, o));
     }
-    __syncthreads();
-    sh[g][cl] = w;
-    if (kMinMax) {
-      shn[g][cl] = wn;
-      shx[g][cl] = wx;
-    }
-    __syncthreads();
   }
-  sum = sh[0][cl];
+  sum = v;                 // the result for channel g of the block (every lane of warp g)
   if (kMinMax) {
-    vmin = shn[0][cl];
-    vmax = shx[0][cl];
+    vmin = vn;
+    vmax = vx;
   }
 }
 
@@ -336,10 +338,11 @@ __device__ __forceinline__ void k_mean_body(int bx, const double* __restrict__ p
   float dummy0, dummy1;
   finalize_channel<false>(psum, nullptr, nullptr, nsb, HD, b, ch, valid, sh, nullptr, nullptr, s, dummy0,
                           dummy1);
-  if (valid && threadIdx.x < 32) {
+  const int och = bx * 32 + (threadIdx.x >> 5);   // warp g finished channel g of the block
+  if (och < B * HD && (threadIdx.x & 31) == 0) {
     const uint16_t m = static_cast<uint16_t>(double_to_bf16_bits(__ddiv_rn(s, static_cast<double>(N))));
-    mean_ws[gch] = m;
-    if (mean_out) mean_out[gch] = m;
+    mean_ws[och] = m;
+    if (mean_out) mean_out[och] = m;
   }
 }
 
@@ -364,7 +367,8 @@ __device__ __forceinline__ void v_stats_body(int bx, const double* __restrict__ 
   double s = 0.0;
   float vmin = 0.f, vmax = 0.f;
   finalize_channel<true>(psum, pmin, pmax, nsb, HD, b, ch, valid, sh, shn, shx, s, vmin, vmax);
-  if (valid && threadIdx.x < 32) {
+  const int och = bx * 32 + (threadIdx.x >> 5);   // warp g finished channel g of the block
+  if (och < B * HD && (threadIdx.x & 31) == 0) {
     const float mean = __double2float_rn(__ddiv_rn(s, static_cast<double>(N)));
     const float amax = fmaxf(__fsub_rn(vmax, mean), __fsub_rn(mean, vmin));
     float scale = 0.f, inv = 0.f;
@@ -372,9 +376,9 @@ __device__ __forceinline__ void v_stats_body(int bx, const double* __restrict__ 
       scale = __fdiv_rn(amax, 448.f);
       inv = __fdiv_rn(448.f, amax);
     }
-    v_mean[gch] = mean;
-    v_scale[gch] = scale;
-    v_inv[gch] = inv;
+    v_mean[och] = mean;
+    v_scale[och] = scale;
+    v_inv[och] = inv;
   }
 }
 
