@@ -14,7 +14,10 @@ value      = attention ops (4*B*H*N^2*D, INT8 QK^T + FP8 PV) per step, all ranks
              inputs resident in HBM, L2 flushed (256 MiB write) between steps,
              per-step CUDA events on the launching stream, max over ranks.
 e2e        = the same metric through the Python API with pinned host inputs:
-             H2D of Q, K, V + the three calls + D2H of the BF16 output, per step.
+             H2D of Q, K, V + the calls + D2H of the BF16 output, every step,
+             pipelined over two buffer sets (copy-in, compute, copy-out on three
+             streams; one device-timed region over all K steps); the one-stream
+             serial figure is reported beside it.
 roofline   = the attention kernel alone: ops / its mean event-timed duration,
              against the INT8/FP8 dense peak derived from the measured BF16 peak.
 cpu_baseline (N=1, rank 0) = the CPU oracle timed on a bounded sample.
@@ -151,6 +154,45 @@ def job_tops(world: int, ops_per_step: float, steps: int, max_total_ms: float) -
     """Whole-job throughput: every rank runs `steps` steps of its own batch
     (replicas), so the job does world * ops * steps in the slowest rank's time."""
     return world * ops_per_step * steps / (max_total_ms / 1e3) / 1e12
+
+
+def pipelined_e2e(torch, n: int, stream, copy_in, compute, copy_out) -> float:
+    """Device milliseconds of n end-to-end steps over two device buffer sets
+    (slot = step & 1): copy_in(slot) (host -> device) runs on one stream,
+    compute(slot) on `stream`, copy_out(slot) (device -> host) on a third, so
+    step i+1's inputs cross PCIe while step i computes.  A slot's inputs are
+    rewritten only after the step two back has computed on them, and its
+    outputs only after they have been copied out.  One pair of events on
+    `stream` brackets the whole region."""
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    new_ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    start, end = new_ev(), new_ev()
+    computed, copied = [None] * n, [None] * n
+    start.record(stream)
+    s_in.wait_event(start)
+    for i in range(n):
+        slot = i & 1
+        if i >= 2:
+            s_in.wait_event(computed[i - 2])
+        with torch.cuda.stream(s_in):
+            copy_in(slot)
+        ready = new_ev()
+        ready.record(s_in)
+        stream.wait_event(ready)
+        if i >= 2:
+            stream.wait_event(copied[i - 2])
+        compute(slot)
+        computed[i] = new_ev()
+        computed[i].record(stream)
+        s_out.wait_event(computed[i])
+        with torch.cuda.stream(s_out):
+            copy_out(slot)
+        copied[i] = new_ev()
+        copied[i].record(s_out)
+    stream.wait_event(copied[n - 1])
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -429,15 +471,16 @@ def run_fp8_linear(args, rank, world, local):
         gemm_us[name] = 1e3 * statistics.mean(e[1 + j].elapsed_time(e[1 + nd + j]) for e in ev)
 
     # e2e: pinned host activations in, BF16 projection outputs back, every step
+    # (serial on one stream, then pipelined over two buffer sets)
     hx = [torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory() for xb, _, _ in host]
-    hout = [torch.empty(d["out"].shape, dtype=torch.bfloat16).pin_memory() for d in dev]
+    hout = [[torch.empty(d["out"].shape, dtype=torch.bfloat16).pin_memory() for d in dev] for _ in range(2)]
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
 
     def e2e_step():
         for d, h in zip(dev, hx):
             d["x"].copy_(h, non_blocking=True)
         step()
-        for d, h in zip(dev, hout):
+        for d, h in zip(dev, hout[0]):
             h.copy_(d["out"], non_blocking=True)
     for _ in range(2):
         e2e_step()
@@ -451,8 +494,34 @@ def run_fp8_linear(args, rank, world, local):
     torch.cuda.synchronize()
     barrier()
     adt.sage_check()
-    e2e_value = job_tops(world, flops, K_steps, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world,
-                                                                "cuda"))
+    e2e_serial = job_tops(world, flops, K_steps, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world,
+                                                                 "cuda"))
+    dev2 = [dict(d, x=torch.empty_like(d["x"]), xq=torch.empty_like(d["xq"]), sx=torch.empty_like(d["sx"]),
+                 out=torch.empty_like(d["out"])) for d in dev]
+    sets = [dev, dev2]
+
+    def copy_in(j):
+        for d, h in zip(sets[j], hx):
+            d["x"].copy_(h, non_blocking=True)
+
+    def compute(j):
+        for d in sets[j]:
+            adt.sage_fp8_quant_rows(d["x"], d["xq"], d["sx"], stream)
+            adt.sage_fp8_linear(d["xq"], d["sx"], d["wq"], d["sw"], d["out"], stream)
+
+    def copy_out(j):
+        for d, h in zip(sets[j], hout[j]):
+            h.copy_(d["out"], non_blocking=True)
+
+    pipelined_e2e(torch, 3, stream, copy_in, compute, copy_out)
+    barrier()
+    e2e_ms = pipelined_e2e(torch, K_steps, stream, copy_in, compute, copy_out)
+    barrier()
+    adt.sage_check()
+    e2e_value = job_tops(world, flops, K_steps, max_over_ranks(e2e_ms, world, "cuda"))
+    last = (K_steps - 1) & 1
+    if not all(torch.equal(h, d["out"].cpu()) for h, d in zip(hout[last], sets[last])):
+        raise RuntimeError("pipelined e2e: the copied-out output differs from the device result")
     h2d = sum(xb.nbytes for xb, _, _ in host)
     d2h = sum(d["out"].numel() * 2 for d in dev)
 
@@ -489,7 +558,9 @@ def run_fp8_linear(args, rank, world, local):
         "kernels_us": {"quant_x": quant_us, "gemm": gemm_us},
         "quant_gbs": x_bytes / (sum(quant_us.values()) / 1e6) / 1e9,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "copy-in, compute and copy-out on three streams, two buffer sets",
+                "serial_value": e2e_serial},
         "gpu_launches": 2 * len(dev) * K_steps,
         "clocks": clocks,
     }
@@ -538,7 +609,7 @@ def main():
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    def quant_qk():
+    def quant_qk(q=q, k=k, buf=buf):
         if nr is None:
             adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
                               buf.workspace, stream)
@@ -547,23 +618,23 @@ def main():
                                        buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
                                        buf.workspace, stream)
 
-    def quant_v():
+    def quant_v(v=v, buf=buf):
         adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
 
     fused = args.quant == "fused" and nr is None
 
-    def quant_qkv():
+    def quant_qkv(q=q, k=k, v=v, buf=buf):
         adt.sage_quant_qkv(q, k, v, buf.shape, 0, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
                            buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
 
-    def quant_all():
+    def quant_all(q=q, k=k, v=v, buf=buf):
         if fused:
-            quant_qkv()
+            quant_qkv(q, k, v, buf)
         else:
-            quant_qk()
-            quant_v()
+            quant_qk(q, k, buf)
+            quant_v(v, buf)
 
-    def attn():
+    def attn(buf=buf):
         adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
                           buf.v_mean, buf.shape, 0.0, buf.out, False, None, stream)
 
@@ -611,14 +682,19 @@ def main():
     value = job_tops(world, ops, K, max_total_ms)
 
     # --------------------------------------------------------------- e2e (host buffers)
+    # Every step copies its Q, K, V in from pinned host memory and its output
+    # back.  Serial: copy in, compute, copy out on one stream.  Pipelined (the
+    # reported figure): two device buffer sets, copies in on one stream, the
+    # calls on another, copies out on a third, so step i+1's inputs cross PCIe
+    # while step i computes; events order each slot's reuse.
     pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
     hq, hk, hv = pin(qb), pin(kb), pin(vb)
-    hout = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+    hout = [torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory() for _ in range(2)]
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for _ in range(2):
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
         quant_all(); attn()
-        hout.copy_(buf.out, non_blocking=True)
+        hout[0].copy_(buf.out, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
     for i in range(K):
@@ -626,12 +702,36 @@ def main():
         e2e_ev[i][0].record(stream)
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
         quant_all(); attn()
-        hout.copy_(buf.out, non_blocking=True)
+        hout[0].copy_(buf.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     adt.sage_check()
-    e2e_value = job_tops(world, ops, K, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, "cuda"))
+    e2e_serial = job_tops(world, ops, K, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, "cuda"))
+
+    buf2 = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=args.q_gran, k_gran=args.k_gran)
+    slots = [(q, k, v, buf), (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), buf2)]
+
+    def copy_in(j):
+        for d, h in zip(slots[j][:3], (hq, hk, hv)):
+            d.copy_(h, non_blocking=True)
+
+    def compute(j):
+        quant_all(*slots[j])
+        attn(slots[j][3])
+
+    def copy_out(j):
+        hout[j].copy_(slots[j][3].out, non_blocking=True)
+
+    pipelined_e2e(torch, 3, stream, copy_in, compute, copy_out)
+    barrier()
+    e2e_ms = pipelined_e2e(torch, K, stream, copy_in, compute, copy_out)
+    barrier()
+    adt.sage_check()
+    e2e_value = job_tops(world, ops, K, max_over_ranks(e2e_ms, world, "cuda"))
+    out_ok = torch.equal(hout[(K - 1) & 1], buf2.out.cpu() if (K - 1) & 1 else buf.out.cpu())
+    if not out_ok:
+        raise RuntimeError("pipelined e2e: the copied-out output differs from the device result")
     h2d = 3 * qb.nbytes
     d2h = buf.out.numel() * buf.out.element_size()
 
@@ -682,7 +782,9 @@ def main():
         "kernels_us": quant_us,
         "quant_gbs": quant_gbs,
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "copy-in, compute and copy-out on three streams, two buffer sets",
+                "serial_value": e2e_serial},
         "gpu_launches": (5 if fused else 7) * K,
         "clocks": clocks,
     }
