@@ -30,7 +30,9 @@ every scale granularity: 64-token blocks, per token, segment-local blocks; the a
 against brute-force FP64 softmax attention; smoothing by the softmax shift
 invariance; closed forms for degenerate inputs; the softmax exp2 against
 numpy's exp2 within its stated error bound and exactly at integers; the fused
-multiply-add against exact rational rounding).  With the exp2 and the FMA
+multiply-add against exact rational rounding; the exponent formed on biased
+scores against exact rationals; the running-max slack by its rule and, with
+the score bias, by brute-force softmax).  With the exp2 and the FMA
 fixed by the contract, the E4M3 codes of P are reproducible; attention parity
 keeps a tolerance for the tensor core's FP32 summation order and the order of
 the row-sum additions.
@@ -53,6 +55,8 @@ INT8_MAX = 127.0
 E4M3_MAX = 448.0
 LOG2E = 1.4426950408889634
 LOG2_P_UNIT = np.float32(math.log2(E4M3_MAX))   # RN32(log2 448), the P scale in the exponent
+S_BIAS = np.float32(12582912.0)  # 1.5 * 2^23: integer scores are carried as the binary32 S + S_BIAS
+MAX_SLACK = np.float32(2.0)      # a raised running max is set this far (exp2 units) above the tile max
 
 
 def npad(n: int) -> int:
@@ -333,7 +337,7 @@ def _identity(x):
 
 
 def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2_alpha, quant_p,
-                 log2_p_unit, two_pass=False):
+                 log2_p_unit, two_pass=False, s_bias=0.0, slack=0.0):
     """Online-softmax attention over 128-key tiles for one (b, h).
 
     S         [R, >= n_keys] float64: exact score numerators (INT32 dot
@@ -350,18 +354,32 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
     quant_p   P quantizer (E4M3 round trip, or identity).
     log2_p_unit  log2 of the P scale folded into the exponent: RN32(log2 448)
               with quantization on, 0 with it off.
+    s_bias    the bias B the scores are carried on (S_BIAS with quantization
+              on: the integer S as the binary32 S + B, exact for |S| < 2^22;
+              0 with it off).
+    slack     how far above the tile max a raised running max is set (MAX_SLACK
+              with quantization on, 0 with it off).
 
     Per tile j (keys j0..j1-1, those >= n_keys excluded):
       t     = rn(S * c)                          scores in the exp2 domain
-      m_new = max(m, max_k t)                    running row max
-      alpha = exp2_alpha(rn(m - m_new))          (0 on the first tile, m = -inf)
+      m_new = rn(max_k t + slack) if max_k t > m else m
+                                                 running row max, an upper bound
+                                                 of every t so far
+      alpha = exp2_alpha(rn(m - m_new))          (0 on the first tile, m = -inf;
+                                                 exactly 1 while m is unchanged)
       e     = rn(log2_p_unit - m_new)
-      y     = exp2(fma(S, c, e))                 = P~ * 448, P~ = exp2(t - m_new)
+      e'    = fma(-B, c, e)                      the exponent offset for biased scores
+      y     = exp2(fma(S + B, c, e'))            = P~ * 448 * 2^-(m_new - max t),
+                                                 P~ = exp2(t - m_new) up to e's rounding
       l     = rn(rn(l * alpha) + rn(sum_k y))    row sum of the unquantized y
-      P8    = quant_p(y)                         E4M3 code of P~ * 448
+      P8    = quant_p(y)                         E4M3 code of y (<= 448)
       acc   = rn(rn(acc * alpha) + rn(P8 @ V))   product sum exact, then rounded
     Epilogue: o = fma(rn(acc * out_mult), rn(1 / l), out_add); the P scale
-    cancels between acc and l.
+    and the slack cancel between acc and l.
+    With B = 0, e' = e and y = exp2(fma(S, c, e)); with B != 0 the single
+    rounding of e' shifts every exponent of a (row, c) pair by the same
+    amount, at most half an ulp of B * c (below 1.5 c, under two units of the
+    integer score).
     two_pass: m is the final row max from the start (alpha = 1 throughout).
     Returns (o [R, D], m [R], l [R]).
     """
@@ -380,13 +398,16 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
         j0, j1 = j * TILE, min(n_keys, (j + 1) * TILE)
         c = col_mult(j0, j1)
         t = rn(S[:, j0:j1] * c)
-        m_new = m if two_pass else np.maximum(m, t.max(axis=1))
+        tmax = t.max(axis=1)
+        m_new = m if two_pass else np.where(tmax > m, rn(tmax + np.float64(slack)), m)
         with np.errstate(invalid="ignore"):
             alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2_alpha(rn(m - m_new)), dtype=np.float64))
         if two_pass:
             alpha = np.ones(R)
         e = rn(log2_p_unit - m_new)
-        y = np.asarray(exp2(fma(S[:, j0:j1], c, e[:, None])), dtype=np.float64)
+        c_full = np.broadcast_to(c, S[:, j0:j1].shape)
+        e_off = np.asarray(fma(np.float64(-s_bias), c_full, e[:, None]), dtype=np.float64)
+        y = np.asarray(exp2(fma(S[:, j0:j1] + np.float64(s_bias), c_full, e_off)), dtype=np.float64)
         l = rn(rn(l * alpha) + rn(y.sum(axis=1)))
         p8 = quant_p(y)
         acc = rn(rn(acc * alpha[:, None]) + rn(p8 @ Vt[:, j0:j1].T))
@@ -423,9 +444,10 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     Score dequant multiplier for query row i and key j, with qs[i] and ks[j]
     the scales of the groups that hold token i of Q and token j of K:
         c = RN32(RN32(qs[i] * ks[j]) * RN32(sm_scale * log2 e)),
-    the P scale 448 enters the exponent as RN32(log2 448) (P8 = E4M3(P~ * 448),
-    with the exponent of P~ * 448 formed by one fused multiply-add), the row
-    sum holds P~ * 448 and the output factor is the V scale itself.
+    the P scale 448 enters the exponent as RN32(log2 448) (P8 = E4M3(y), y =
+    P~ * 448 below the slack of the running max, with the exponent formed by
+    one fused multiply-add on the biased score S + S_BIAS), the row sum holds y
+    and the output factor is the V scale itself.
     sm_scale None or <= 0 means 1/sqrt(D).
     rows: optional query-row indices (< N) to evaluate; heads: optional list of
     (b, h) pairs.  Returns float32 [B, R, H, D] (unevaluated heads stay 0),
@@ -452,23 +474,27 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
             return rn32(rn32(qs[:, None].astype(np.float64) * kk[None, :]) * np.float64(sl2e))
 
         Vt = e4m3_decode(v_codes_t[b, h, :, :N])
+        assert np.abs(S).max(initial=0) < 2.0 ** 22          # S + S_BIAS is an exact binary32
         o, m, l = _attend_rows(S, col_mult, Vt, v_scale[b, h].astype(np.float64),
                                v_mean[b, h].astype(np.float64), N, rn32, fma32, exp2_contract,
-                               _exp2_alpha, _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass)
+                               _exp2_alpha, _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass,
+                               s_bias=S_BIAS, slack=MAX_SLACK)
         out[b, :, h, :] = o
         lse[b, h] = rn32((m + np.log2(l) - math.log2(E4M3_MAX)) * math.log(2.0))
     return (out, lse) if want_lse else out
 
 
 def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
-                     smooth_v=True, heads=None):
+                     smooth_v=True, heads=None, s_bias=0.0, slack=0.0):
     """The same tile loop with quantization OFF, all in FP64.
 
     q, k, v: float64 [B, N, H, D].  Scores are exact FP64 dot products, the
     multiplier is sm_scale * log2 e, P is not quantized (p_unit 1), V is
     centred by its FP64 mean (smooth_v) and K by its FP64 mean (smooth_k).
-    Used to pin the tile loop, the rescaling and the smoothing algebra against
-    brute-force softmax attention.  Returns float64 [B, R, H, D].
+    s_bias, slack: the score bias and the running-max slack of the quantized
+    loop, which must cancel.  Used to pin the tile loop, the rescaling, the
+    biased exponent and the smoothing algebra against brute-force softmax
+    attention.  Returns float64 [B, R, H, D].
     """
     B, _, H, D = q.shape
     if sm_scale is None or sm_scale <= 0:
@@ -486,7 +512,8 @@ def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
         mean = V.mean(axis=0) if smooth_v else np.zeros(D)
         S = Q @ K.T
         o, _, _ = _attend_rows(S, lambda j0, j1: c, (V - mean).T, np.ones(D), mean,
-                               N, _identity, _fma_exact, np.exp2, np.exp2, _identity, 0.0)
+                               N, _identity, _fma_exact, np.exp2, np.exp2, _identity, 0.0,
+                               s_bias=s_bias, slack=slack)
         out[b, :, h, :] = o
     return out
 

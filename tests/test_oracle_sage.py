@@ -165,6 +165,57 @@ def test_tile_loop_quant_off_equals_brute_force(B, N, H, D):
     ref = so.attn_exact_fp64(q, k, v, N)
     got = so.attn_unquantized(q, k, v, N)
     assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    # The score bias and the running-max slack cancel: the same loop with the
+    # quantized path's B = 1.5 * 2^23 and slack 2 (FP64 rounding of the biased
+    # product and offset, ~2^-52 * B * c, is the only difference).
+    got_b = so.attn_unquantized(q, k, v, N, s_bias=float(so.S_BIAS), slack=float(so.MAX_SLACK))
+    assert np.abs(got_b - ref).max() <= 1e-7 * max(1.0, np.abs(ref).max())
+
+
+def test_biased_exponent_is_one_rounding_of_the_offset():
+    """u = fma(S + B, c, e') with e' = fma(-B, c, e): within half an ulp of e'
+    plus half an ulp of u of the exact S * c + e (rationals), for integer
+    scores up to the INT8 maximum 127^2 * 128 and multipliers over 18 binades.
+    The wrong-sign offset (e' = fma(+B, c, e)) is off by 2 B c."""
+    rng = np.random.default_rng(31)
+    n = 300
+    smax = 127 * 127 * 128
+    S = np.concatenate([[0, smax, -smax, 1, -1], rng.integers(-smax, smax + 1, n - 5)]).astype(np.float64)
+    c = np.float32(2.0) ** rng.uniform(-20, -2, n).astype(np.float32)
+    c = (c * np.float32(1) + np.float32(0) * c).astype(np.float32)
+    e = rng.uniform(-40, 9, n).astype(np.float32)
+    B = so.S_BIAS
+    e_off = nm.fma32(-B, c, e)
+    u = nm.fma32(S + np.float64(B), c, e_off)
+    for i in range(n):
+        exact = Fraction(int(S[i])) * Fraction(float(c[i])) + Fraction(float(e[i]))
+        bound = Fraction(float(np.spacing(np.abs(e_off[i])))) / 2 + Fraction(float(np.spacing(np.abs(u[i])))) / 2
+        assert abs(Fraction(float(u[i])) - exact) <= bound, i
+    wrong = nm.fma32(S + np.float64(B), c, nm.fma32(B, c, e))
+    assert np.all(np.abs(wrong.astype(np.float64) - u) >= 1.9 * float(B) * c.astype(np.float64))
+
+
+def test_running_max_slack_rule():
+    """One row, three 128-key tiles with maxima 5, 6.5 and 10 (multiplier 1):
+    the first tile sets m = 5 + 2, the second (6.5 <= 7) leaves it, the third
+    raises it to 12; the output is the brute-force softmax either way, and an
+    unchanged m rescales by exactly 1 in the contract's exp2."""
+    rng = np.random.default_rng(32)
+    n = 384
+    S = rng.uniform(-4, 4, (1, n))
+    S[0, 17], S[0, 200], S[0, 300] = 5.0, 6.5, 10.0
+    V = rng.standard_normal((4, n))
+    args = (S, lambda j0, j1: 1.0, V, np.ones(4), np.zeros(4), n, so._identity, so._fma_exact,
+            np.exp2, np.exp2, so._identity, 0.0)
+    o, m, _ = so._attend_rows(*args, slack=2.0)
+    assert m[0] == 12.0
+    w = np.exp2(S[0] - S[0].max())
+    assert np.allclose(o[0], (w / w.sum()) @ V.T, rtol=0, atol=1e-12)
+    S2 = S.copy()
+    S2[0, 300] = 7.0                                   # equal to m: no raise
+    _, m2, _ = so._attend_rows(S2, *args[1:], slack=2.0)
+    assert m2[0] == 7.0
+    assert so._exp2_alpha(np.float32(0.0)) == np.float32(1.0)
 
 
 def test_k_smoothing_is_softmax_invariant():
@@ -221,15 +272,20 @@ def test_closed_form_dominant_key():
     dec = dec_all[200]
     # The other keys keep the exact softmax weight 1 - w200 of the dequantized
     # scores (E4M3 rounding of their P moves it by < 10%); and key 200's code is
-    # E4M3(y) = 448 while the row sum holds y itself, whose exp2 is within the
-    # quadratic's 1.963e-3, so the centred output moves by up to that ratio.
+    # E4M3(y) = 112 (the running max sits 2 above its score) while the row sum
+    # holds y itself, whose exp2 is within the quadratic's 1.963e-3 and whose
+    # exponent carries the offset's rounding (half an ulp of B * c + |e|), so
+    # the centred output moves by up to that ratio.
     qd = it["q_codes"][0, 0, 5].astype(np.float64) * it["q_scale"][0, 0, 0]
     kd = it["k_codes"][0, 0, :N].astype(np.float64) * np.repeat(it["k_scale"][0, 0], 64)[:N, None]
     s = kd @ qd / 8.0
     w = np.exp(s - s.max())
     w /= w.sum()
     spread = np.abs(dec_all - dec).max(axis=0)
-    tol = 1.1 * (1 - w[200]) * spread + 1.97e-3 * np.abs(dec - it["v_mean"][0, 0]) + 1e-6
+    c = nm.rn32(nm.rn32(np.float64(it["q_scale"][0, 0, 0]) * it["k_scale"][0, 0, 3])
+                * np.float64(so.exp2_scale(so.default_sm_scale(D))))
+    off = math.log(2) * float(np.spacing(np.float32(float(so.S_BIAS) * float(c) + 64.0))) / 2
+    tol = 1.1 * (1 - w[200]) * spread + (1.963e-3 + off) * np.abs(dec - it["v_mean"][0, 0]) + 1e-6
     assert w[200] > 0.999
     assert np.all(np.abs(o[0, 5, 0] - dec) <= tol)
 
@@ -300,17 +356,19 @@ def test_running_max_with_large_logit_gap():
     o, it = _pipeline(q, k, v)
     assert np.all(np.isfinite(o))
     dec = nm.e4m3_decode(it["v_codes_t"][0, 0, :, 10]) * it["v_scale"][0, 0] + it["v_mean"][0, 0]
-    # The dominant key's exponent is S*c - RN(S*c) + (RN(log2 448 - m) - (log2 448 - m)):
-    # off by at most one FP32 ulp of the row max m (here ~1150), and its exp2 is
-    # within the quadratic's 1.963e-3, while its code is 448 either way: the centred
-    # output moves by up to ln2 * ulp(m) + 1.963e-3 relative.
+    # The dominant key's exponent is S*c - RN(S*c) + (RN(log2 448 - m) - (log2 448 - m))
+    # plus the offset's rounding: off by at most one FP32 ulp of the row max m (here
+    # ~1150) and half an ulp of B * c + |e|, and its exp2 is within the quadratic's
+    # 1.963e-3, while its code is 112 either way: the centred output moves by up to
+    # ln2 * (ulp(m) + ulp(B c + |e|) / 2) + 1.963e-3 relative.
     S = it["q_codes"][0, 0, 5].astype(np.float64) @ it["k_codes"][0, 0, 10].astype(np.float64)
     c = nm.rn32(nm.rn32(np.float64(it["q_scale"][0, 0, 0]) * it["k_scale"][0, 0, 0])
                 * np.float64(so.exp2_scale(so.default_sm_scale(D))))
     m = nm.rn32(S * np.float64(c))
     assert m > 512
     centred = np.abs(dec - it["v_mean"][0, 0])                  # the part scaled by P8 / l
-    tol = (2 * np.spacing(np.float32(m)) + 1.97e-3) * centred + 1e-6
+    off = float(np.spacing(np.float32(float(so.S_BIAS) * float(c) + 2 * float(m)))) / 2
+    tol = (math.log(2) * (np.spacing(np.float32(m)) + off) + 1.963e-3) * centred + 1e-6
     assert np.all(np.abs(o[0, 5, 0] - dec) <= tol)
 
 
