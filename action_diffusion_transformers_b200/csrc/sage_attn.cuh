@@ -47,6 +47,7 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSBiasBits = 0x4B400000u;   // S accumulates onto these bits
 constexpr float kSBias = 12582912.0f;          // their float value, 1.5 * 2^23
 constexpr float kLog2P8 = 8.8073549220576041f; // log2(448): the P scale, folded into the exponent
+constexpr float kMaxSlack = 2.0f;                // a raised running max sits this far above the tile max
 
 template <int D>
 struct AttnSmem {
@@ -98,15 +99,17 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
   return __int2float_rn(static_cast<int>(s));
 }
 
-// The contract's exponentials for 32 of this thread's keys (biased scores s as
-// loaded from TMEM; valid counts from the first of them): u = RN(S * c + e) with e = RN(log2 448 - m_new) (one fused
-// multiply-add), y = exp2_fixed_x2(u) = P~ * 448 -> E4M3 code; the row sum
-// accumulates y.  Every step is a binary32 operation with fixed rounding, so y
-// and its code equal the oracle's bit for bit.  kClamp: some u of this warp's
-// tile may be below -126.  pk[w] holds the codes of keys 4w .. 4w+3.
-// cmul(p) gives the multipliers c of the quarter's keys 2p and 2p+1.
+// The contract's exponentials for 32 of this thread's keys (biased scores
+// Sb = S + 1.5 * 2^23 as loaded from TMEM; valid counts from the first of
+// them): u = RN(Sb * c + e') with e' = RN(e - 1.5 * 2^23 * c) and
+// e = RN(log2 448 - m_new) (one fused multiply-add per key), y = exp2_fixed_x2(u)
+// -> E4M3 code; the row sum accumulates y.  Every step is a binary32 operation
+// with fixed rounding, so y and its code equal the oracle's bit for bit.
+// kClamp: some u of this warp's tile may be below -126.  pk[w] holds the codes
+// of keys 4w .. 4w+3.  cmul(p) gives the multipliers c and offsets e' of the
+// quarter's keys 2p and 2p+1.
 template <bool kMasked, bool kClamp, class CMul>
-__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const CMul& cmul, f32x2_t e2, int valid,
+__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const CMul& cmul, int valid,
                                                 const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
   // Stage-major over 8 pairs at a time: every step is issued for 8 independent
   // pairs before the next step, so consecutive instructions do not depend on
@@ -117,10 +120,9 @@ __device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const C
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int j = 8 * h8 + i;
-      u[i] = x2_sub(x2_pack(s[2 * j], s[2 * j + 1]), k.round);   // exact integer S (the S bias is 1.5 * 2^23 too)
+      const auto mo = cmul(j);
+      u[i] = x2_fma(x2_pack(s[2 * j], s[2 * j + 1]), mo.c, mo.off);
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) u[i] = x2_fma(u[i], cmul(8 * h8 + i), e2);
     if (kClamp) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -178,34 +180,43 @@ __device__ __forceinline__ void chunk_minmax(const uint32_t (&a)[32], int valid,
              fmaxf(w[9], w[10]));
 }
 
-// One multiplier for every key of a quarter (its 64-key half shares one K scale).
-struct UniformMul {
-  f32x2_t c2;
-  __device__ __forceinline__ f32x2_t operator()(int) const { return c2; }
+// Multipliers c and exponent offsets e' = RN(e - 1.5 * 2^23 * c) of a key pair.
+struct MulOff {
+  f32x2_t c, off;
 };
 
-// Per-key multipliers c = RN(RN(qs * ks_j) * sl2e): lane L holds ks of key
-// 32 * quarter + L in kq, and a shuffle brings it to every row.
+// One multiplier and offset for every key of a quarter (its 64-key half shares
+// one K scale).
+struct UniformMul {
+  MulOff mo;
+  __device__ __forceinline__ MulOff operator()(int) const { return mo; }
+};
+
+// Per-key multipliers c = RN(RN(qs * ks_j) * sl2e) and their offsets: lane L
+// holds ks of key 32 * quarter + L in kq, and a shuffle brings it to every row.
 struct KeyMul {
-  f32x2_t qs2, sl2e2;
+  f32x2_t qs2, sl2e2, e2;
   float kq;
-  __device__ __forceinline__ f32x2_t operator()(int p) const {
+  __device__ __forceinline__ MulOff operator()(int p) const {
     const float k0 = __shfl_sync(0xFFFFFFFFu, kq, 2 * p);
     const float k1 = __shfl_sync(0xFFFFFFFFu, kq, 2 * p + 1);
-    return x2_mul(x2_mul(x2_pack(__float_as_uint(k0), __float_as_uint(k1)), qs2), sl2e2);
+    const f32x2_t c = x2_mul(x2_mul(x2_pack(__float_as_uint(k0), __float_as_uint(k1)), qs2), sl2e2);
+    return MulOff{c, x2_fma(x2_splat(-kSBias), c, e2)};
   }
 };
 
-struct HalfMuls {      // keys 0-63 use c0, keys 64-127 use c1
-  float c0, c1;
-  __device__ __forceinline__ UniformMul operator()(int qq) const { return UniformMul{x2_splat(qq < 2 ? c0 : c1)}; }
+struct HalfMuls {      // keys 0-63 use (c0, off0), keys 64-127 (c1, off1)
+  float c0, c1, off0, off1;
+  __device__ __forceinline__ UniformMul operator()(int qq) const {
+    return UniformMul{MulOff{x2_splat(qq < 2 ? c0 : c1), x2_splat(qq < 2 ? off0 : off1)}};
+  }
 };
 
 struct KeyMuls {       // per-key scales of the tile's four 32-key quarters
-  float qs, sl2e;
+  float qs, sl2e, e;
   const float (&kq)[4];
   __device__ __forceinline__ KeyMul operator()(int qq) const {
-    return KeyMul{x2_splat(qs), x2_splat(sl2e), kq[qq]};
+    return KeyMul{x2_splat(qs), x2_splat(sl2e), x2_splat(e), kq[qq]};
   }
 };
 
@@ -214,9 +225,8 @@ struct KeyMuls {       // per-key scales of the tile's four 32-key quarters
 // the row's 128B-swizzled P line (16-byte chunk q of row r lives at q ^ (r & 7)).
 // kSlow: masked keys or clamped exponents.  muls(qq) gives quarter qq's multipliers.
 template <bool kSlow, class Muls>
-__device__ __forceinline__ void exp_pass(uint32_t taddr, const Muls& muls, float e, int valid,
+__device__ __forceinline__ void exp_pass(uint32_t taddr, const Muls& muls, int valid,
                                          const Exp2Consts& ek, f32x2_t (&lsum)[4], uint8_t* prow, int row) {
-  const f32x2_t e2 = x2_splat(e);
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) {
     uint32_t cur[32];
@@ -224,7 +234,7 @@ __device__ __forceinline__ void exp_pass(uint32_t taddr, const Muls& muls, float
     tmem_wait_ld();
     reg_fence(cur);
     uint32_t pk[8];
-    softmax_quarter<kSlow, kSlow>(cur, muls(qq), e2, valid - 32 * qq, ek, lsum, pk);
+    softmax_quarter<kSlow, kSlow>(cur, muls(qq), valid - 32 * qq, ek, lsum, pk);
     *reinterpret_cast<uint4*>(prow + ((2 * qq) ^ (row & 7)) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     *reinterpret_cast<uint4*>(prow + ((2 * qq + 1) ^ (row & 7)) * 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
   }
@@ -266,7 +276,7 @@ __device__ __forceinline__ f32x2_t keywise_exp_pass(uint32_t taddr, float qs, fl
   for (int i = 0; i < 4; ++i) kq[i] = ks[32 * i + lane];
   const Exp2Consts ek;
   f32x2_t lsum[4] = {0, 0, 0, 0};
-  exp_pass<true>(taddr, KeyMuls{qs, sl2e, kq}, e, valid, ek, lsum, prow, row);
+  exp_pass<true>(taddr, KeyMuls{qs, sl2e, e, kq}, valid, ek, lsum, prow, row);
   return x2_add(x2_add(lsum[0], lsum[1]), x2_add(lsum[2], lsum[3]));
 }
 
@@ -322,16 +332,20 @@ struct SoftmaxTile {
       }
       tmax = __fmul_rn(__fsub_rn(fmaxf(mx[0], mx[1]), kSBias), c0);
       if (valid > 64) tmax = fmaxf(tmax, __fmul_rn(__fsub_rn(fmaxf(mx[2], mx[3]), kSBias), c1));
-      smin0 = __fsub_rn(fminf(mn[0], mn[1]), kSBias);
-      smin1 = __fsub_rn(fminf(mn[2], mn[3]), kSBias);
+      smin0 = fminf(mn[0], mn[1]);       // biased
+      smin1 = fminf(mn[2], mn[3]);
     }
-    const float m_new = fmaxf(m, tmax);
+    // A raised running max sits kMaxSlack above the tile max, so that later
+    // tiles rarely move it (and alpha is exactly 1 while it stays).
+    const float m_new = tmax > m ? __fadd_rn(tmax, kMaxSlack) : m;
     const float alpha = exp2_fixed5(__fsub_rn(m, m_new));
     const float e = __fsub_rn(kLog2P8, m_new);
+    const float off0 = __fmaf_rn(-kSBias, c0, e);
+    const float off1 = __fmaf_rn(-kSBias, c1, e);
     // u is monotone in S (c > 0), so the smallest u of a block is its min S's;
     // clamping is the identity unless that is below -126.
     const bool clamp = kKeywise ||
-                       __any_sync(0xFFFFFFFFu, fminf(__fmaf_rn(smin0, c0, e), __fmaf_rn(smin1, c1, e)) < kExp2Min);
+                       __any_sync(0xFFFFFFFFu, fminf(__fmaf_rn(smin0, c0, off0), __fmaf_rn(smin1, c1, off1)) < kExp2Min);
     // P is single-buffered in shared memory: PV_{j-1} (issued right after QK_j)
     // must have read it before this tile's codes are written.
     if (j > 0 && !warp_wait(&bars[kBarPVDone], static_cast<uint32_t>(j - 1) & 1, abort_flag, tmo)) return false;
@@ -339,9 +353,9 @@ struct SoftmaxTile {
     if constexpr (kKeywise)
       lsum[0] = keywise_exp_pass(ts, qs, sl2e, ks + j * kBN, e, valid, prow, row);
     else if (valid >= kBN && !clamp)
-      exp_pass<false>(ts, HalfMuls{c0, c1}, e, kBN, ek, lsum, prow, row);
+      exp_pass<false>(ts, HalfMuls{c0, c1, off0, off1}, kBN, ek, lsum, prow, row);
     else
-      exp_pass<true>(ts, HalfMuls{c0, c1}, e, valid, ek, lsum, prow, row);
+      exp_pass<true>(ts, HalfMuls{c0, c1, off0, off1}, valid, ek, lsum, prow, row);
     // Re-seed S with the bias for the next tile's MMA, then release the buffer.
     tmem_fill64(ts, kSBiasBits);
     tmem_fill64(ts + 64, kSBiasBits);
