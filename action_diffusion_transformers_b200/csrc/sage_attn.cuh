@@ -11,7 +11,9 @@
 // S is accumulated onto the integer 0x4B400000 (the bits of 1.5 * 2^23) that
 // the softmax warps write into the S columns before each QK^T MMA: read as a
 // float, a loaded S word is then exactly 1.5 * 2^23 + S (|S| <= 127^2 * D <
-// 2^22), so one exact subtraction converts it, two at a time with f32x2.
+// 2^22), and the exponent is formed from it directly: u = fma(S + 1.5 * 2^23,
+// c, e') with the offset e' = fma(-1.5 * 2^23, c, e) formed once per row and
+// 64-key half.
 //   warp 4     producer: one thread issues TMA tile loads (Q once; K and V
 //              tiles into 2-stage rings).
 //   warp 5     MMA: allocates TMEM; one thread issues

@@ -223,13 +223,16 @@ SAGE_API sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_
  * out: out   [B, N, H, D], BF16 (out_fp32 == 0) or FP32 (out_fp32 != 0).
  *      lse   f32 [B, H, N] natural-log softmax denominator, or NULL.
  * Per 128-row query tile and 128-key tile: S = Qc Kc^T exactly in INT32 on the
- * tensor cores; t = S * c in FP32 with c = RN(RN(qs_i * ks_j) * RN(sm_scale *
+ * tensor cores; t = RN(S * c) with c = RN(RN(qs_i * ks_j) * RN(sm_scale *
  * log2 e)), qs_i / ks_j the scales of the groups holding query i / key j;
- * running row max m;
- * P~ = exp2(t - m) in [0, 1]; l accumulates unquantized P~; P8 = E4M3(P~*448);
+ * running row max m, set to RN(max t + 2) when a tile's max exceeds it;
+ * y = exp2(RN((S + B) * c + e')) with B = 1.5 * 2^23, e = RN(log2 448 - m)
+ * and e' = RN(e - B * c), exp2 a fixed binary32 algorithm (Cody-Waite split,
+ * quadratic, exponent-field add); l accumulates y; P8 = E4M3(y) (<= 448);
  * O_acc = O_acc * exp2(m_old - m_new) + P8 V8 (FP8 MMA, FP32 accumulation);
- * O = O_acc * (v_scale/448) / l + v_mean.  Keys >= N are masked.  Matches the
- * contract within tolerance (hardware exp2 and MMA summation order).
+ * O = RN(O_acc * v_scale) * RN(1 / l) + v_mean.  Keys >= N are masked.  The
+ * E4M3 codes of P are the contract's bit for bit; O matches the contract
+ * within the tensor core's FP32 summation order and the row-sum order.
  */
 SAGE_API sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale,
                           const int8_t* k_codes, const float* k_scale,
