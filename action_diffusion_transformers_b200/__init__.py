@@ -264,3 +264,19 @@ class Buffers:
         sage_attn_fwd(self.q_codes, self.q_scale, self.k_codes, self.k_scale, self.v_codes_t, self.v_scale,
                       self.v_mean, self.shape, sm_scale, self.out, self.out_fp32, self.lse, stream)
         return self.out
+
+    def capture(self, q, k, v, sm_scale=0.0, v_shape=None, normrope=None):
+        """The launches of run() on these tensors, captured once into a CUDA
+        graph; graph.replay() then re-runs them on whatever q, k, v hold, with
+        less launch overhead between the kernels.  The calls run once eagerly
+        first (on a side stream) so that every one-time setup happens outside
+        the capture."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.run(q, k, v, sm_scale, side, v_shape, normrope)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            self.run(q, k, v, sm_scale, side, v_shape, normrope)
+        return graph

@@ -11,8 +11,10 @@ BF16 NHD; synthetic, seeded).  Prints ONE JSON line (rank 0).
 
 value      = attention ops (4*B*H*N^2*D, INT8 QK^T + FP8 PV) per step, all ranks,
              / device time of the whole step (quant + attention), in TOPS;
-             inputs resident in HBM, L2 flushed (256 MiB write) between steps,
-             per-step CUDA events on the launching stream, max over ranks.
+             the step's launches replayed as one CUDA graph (eager launches:
+             eager_value); inputs resident in HBM, L2 flushed (256 MiB write)
+             between steps, per-step CUDA events on the launching stream, max
+             over ranks.
 e2e        = the same metric through the Python API with pinned host inputs:
              H2D of Q, K, V + the calls + D2H of the BF16 output, every step,
              pipelined over two buffer sets (copy-in, compute, copy-out on three
@@ -609,34 +611,35 @@ def main():
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    def quant_qk(q=q, k=k, buf=buf):
+    def quant_qk(q=q, k=k, buf=buf, st=None):
+        st = st or stream
         if nr is None:
             adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                              buf.workspace, stream)
+                              buf.workspace, st)
         else:
             adt.sage_quant_qk_normrope(q, k, buf.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
                                        buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                                       buf.workspace, stream)
+                                       buf.workspace, st)
 
-    def quant_v(v=v, buf=buf):
-        adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
+    def quant_v(v=v, buf=buf, st=None):
+        adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or stream)
 
     fused = args.quant == "fused" and nr is None
 
-    def quant_qkv(q=q, k=k, v=v, buf=buf):
+    def quant_qkv(q=q, k=k, v=v, buf=buf, st=None):
         adt.sage_quant_qkv(q, k, v, buf.shape, 0, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                           buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, stream)
+                           buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or stream)
 
-    def quant_all(q=q, k=k, v=v, buf=buf):
+    def quant_all(q=q, k=k, v=v, buf=buf, st=None):
         if fused:
-            quant_qkv(q, k, v, buf)
+            quant_qkv(q, k, v, buf, st)
         else:
-            quant_qk(q, k, buf)
-            quant_v(v, buf)
+            quant_qk(q, k, buf, st)
+            quant_v(v, buf, st)
 
-    def attn(buf=buf):
+    def attn(buf=buf, st=None):
         adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
-                          buf.v_mean, buf.shape, 0.0, buf.out, False, None, stream)
+                          buf.v_mean, buf.shape, 0.0, buf.out, False, None, st or stream)
 
     def barrier():
         if world > 1:
@@ -669,16 +672,43 @@ def main():
         e[3].record(stream)
     torch.cuda.synchronize()
     barrier()
+    adt.sage_check()
+    eager_out = buf.out.clone()
+
+    # The same launches captured once into a CUDA graph and replayed: the
+    # headline value (the per-kernel times and the roofline come from the
+    # eager loop above, whose events sit between the launches).
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        quant_all(st=side)
+        attn(st=side)
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        gev[i][0].record(stream)
+        graph.replay()
+        gev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
     clocks = sampler.stop()
     adt.sage_check()
+    if not torch.equal(buf.out, eager_out):
+        raise RuntimeError("the graph replay's output differs from the eager step's")
 
     step_ms = [e[0].elapsed_time(e[3]) for e in ev]
     quant_ms = [e[0].elapsed_time(e[2]) for e in ev]
     qk_ms = None if fused else [e[0].elapsed_time(e[1]) for e in ev]
     v_ms = None if fused else [e[1].elapsed_time(e[2]) for e in ev]
     at_ms = [e[2].elapsed_time(e[3]) for e in ev]
-    max_total_ms = max_over_ranks(sum(step_ms), world, "cuda")
     ops = w.attn_ops
+    eager_value = job_tops(world, ops, K, max_over_ranks(sum(step_ms), world, "cuda"))
+    max_total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev), world, "cuda")
     value = job_tops(world, ops, K, max_total_ms)
 
     # --------------------------------------------------------------- e2e (host buffers)
@@ -786,6 +816,8 @@ def main():
                 "overlap": "copy-in, compute and copy-out on three streams, two buffer sets",
                 "serial_value": e2e_serial},
         "gpu_launches": (5 if fused else 7) * K,
+        "launch": "the step's launches as one CUDA graph, replayed (eager launches: eager_value)",
+        "eager_value": eager_value,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
