@@ -23,7 +23,7 @@ e2e        = the same metric through the Python API with pinned host inputs:
 roofline   = the attention kernel alone: ops / its mean event-timed duration,
              against the INT8/FP8 dense peak derived from the measured BF16 peak.
 cpu_baseline (N=1, rank 0) = the CPU oracle timed on a bounded sample.
---impl reference runs the oracle (the reference arm of this build) instead.
+--impl reference runs the CPU oracle (the reference arm) instead.
 Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
 (replicas, weak scaling, no collective on the data path).
 """
@@ -785,7 +785,7 @@ def main():
                      "quant_v": v_bytes / (statistics.mean(v_ms) / 1e3) / 1e9, "peak_hbm_gbs": peaks["hbm_gbs"]}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # about 10-30 s of CPU work on the GPU machine's host: 4 heads, 2^26 (query row, key) pairs
+        # about 10-30 s of CPU work on the host: 4 heads, 2^26 (query row, key) pairs
         heads = min(4, w.H)
         rows = max(1, min(w.N, (1 << 26) // (heads * w.N)))
         o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads, args.q_gran, args.k_gran, nr_host)
