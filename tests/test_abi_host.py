@@ -149,3 +149,56 @@ def test_fp8_linear_validation(adt):
     assert L.sage_fp8_linear(FAKE, FAKE, FAKE + 4, FAKE, 16, 16, 32, FAKE, 0, None) == 3
     if not _gpu_present():
         assert L.sage_fp8_linear(FAKE, FAKE, FAKE, FAKE, 16, 16, 32, FAKE, 0, None) == 4
+
+
+def _qkv(adt, shape, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, vts=0, qc=FAKE, qs=FAKE, kc=FAKE, ks=FAKE, km=None, vc=FAKE, vs=FAKE, vm=FAKE,
+             ws=0x100000, wsb=1 << 40)
+    a.update(over)
+    return adt._lib.sage_quant_qkv(a["q"], a["k"], a["v"], shape, a["vts"], a["qc"], a["qs"], a["kc"], a["ks"],
+                                   a["km"], a["vc"], a["vs"], a["vm"], a["ws"], a["wsb"], None)
+
+
+def test_quant_qkv_validation(adt):
+    """The one-call quantization checks its shape, V's token stride, every
+    pointer and the workspace before any CUDA call."""
+    assert _qkv(adt, adt.make_shape(1, 256, 2, 96)) == 2          # unsupported head dim
+    assert _qkv(adt, adt.make_shape(1, 0, 2, 64)) == 1            # empty sequence
+    s = adt.make_shape(1, 256, 2, 64)
+    assert _qkv(adt, s, vts=100) == 1                             # V token stride below H*D
+    assert _qkv(adt, s, vts=132) == 3                             # V token stride not a multiple of 8
+    for name in ("q", "k", "v", "qc", "qs", "kc", "ks", "vc", "vs", "vm"):
+        assert _qkv(adt, s, **{name: None}) == 1, name
+    assert _qkv(adt, s, km=FAKE + 2) == 3                         # k_mean alignment
+    assert _qkv(adt, s, ws=None) == 6
+    assert _qkv(adt, s, wsb=16) == 6
+    assert b"workspace" in adt._lib.sage_last_error()
+    if not _gpu_present():
+        assert _qkv(adt, s) == 4                                  # valid: stops at the device lookup
+        assert _qkv(adt, s, vts=256) == 4                         # a strided V view is valid too
+
+
+def test_quant_qk_static_validation(adt):
+    """The allocation-free variant validates like sage_quant_qk and refuses
+    shapes whose scratch exceeds its built-in array."""
+    lib = adt._lib
+    s = adt.make_shape(1, 256, 2, 64)
+    args = [FAKE, FAKE, s, FAKE, FAKE, FAKE, FAKE, None, None]
+    assert lib.sage_quant_qk_static(*args[:2], adt.make_shape(1, 256, 2, 96), *args[3:]) == 2
+    for i in (0, 1, 3, 4, 5, 6):
+        bad = list(args)
+        bad[i] = None
+        assert lib.sage_quant_qk_static(*bad) == 1, i
+    bad = list(args)
+    bad[7] = FAKE + 2
+    assert lib.sage_quant_qk_static(*bad) == 3
+    big = adt.make_shape(2, 55296, 32, 128)                       # FP64 partial sums far above 8 MiB
+    assert lib.sage_quant_qk_static(FAKE, FAKE, big, FAKE, FAKE, FAKE, FAKE, None, None) == 6
+    assert b"scratch" in lib.sage_last_error()
+
+
+def test_selftest_timeout_range(adt):
+    """The bounded-wait self-test accepts only timeouts in (0, 10 s]."""
+    for bad in (0, -5, 10_000_000_001):
+        assert adt._lib.sage_selftest_wait_timeout(bad, None) == 1
+        assert b"timeout" in adt._lib.sage_last_error()
