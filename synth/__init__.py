@@ -12,7 +12,7 @@ stated configurations, the pages give neither):
                                      joint block; K offsets ~N(0, 4^2) plus 2%
                                      outlier channels x8; V offsets ~N(0, 1)
 * mid_video  B=1 H=24 N=16384 D=128  distributions as action_dit
-* long_video B=1 H=32 N=55296 D=128  31 latent frames x 56 x 32 tokens; K offsets
+* long_video B=1 H=32 N=55296 D=128  the configuration's token count; K offsets
                                      ~N(0, 4^2); 1% heavy-tail rows, Student-t(3)
 * ragged     B=1 H=24 N=20480 D=128  4 concatenated streams (text 512, video
                                      18432, video_cond 1504, action+state 32) given
