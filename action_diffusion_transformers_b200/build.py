@@ -20,8 +20,17 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsage.so")
 SOURCES = [os.path.join(CSRC, "sage_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sage_ptx.cuh", "sage_quant.cuh", "sage_attn.cuh")] + [
-    os.path.join(INCLUDE, "sage.h")]
+
+
+def deps() -> list:
+    """Every file the library is built from: all sources and headers under
+    csrc/ and include/ (so an edit to any of them triggers a rebuild)."""
+    out = []
+    for d in (CSRC, INCLUDE):
+        for name in sorted(os.listdir(d)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                out.append(os.path.join(d, name))
+    return out
 
 
 def nvcc() -> str:
@@ -35,7 +44,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in DEPS)
+    return all(os.path.getmtime(d) <= t for d in deps())
 
 
 def build(verbose: bool = False, force: bool = False) -> str:

@@ -351,7 +351,9 @@ unsigned char* g_qk_static_ptr[kMaxDevices];
 std::mutex g_qk_static_mu;
 
 // Device address of g_qk_static_scratch on the current device (looked up once
-// per device; host code only holds a stand-in for the array's name).
+// per device; host code only holds a stand-in for the array's name).  The
+// address is kept for the life of the process, so it is only valid while the
+// device's primary context is the one it was looked up in (no device reset).
 sage_status qk_static_scratch(int dev, unsigned char** out) {
   std::lock_guard<std::mutex> lock(g_qk_static_mu);
   if (!g_qk_static_ptr[dev]) {

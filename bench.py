@@ -1,13 +1,15 @@
 #!/usr/bin/env python
 """Benchmark of the quantized-attention hot path on B200.
 
-One step = sage_quant_qk + sage_quant_v + sage_attn_fwd over one batch of the
-action-DiT joint-block workload (B=2 CFG cond/uncond, H=24, N=4096, D=128,
-BF16 NHD; synthetic, seeded).  Prints ONE JSON line (rank 0).
+One step = sage_quant_qkv (K/V smoothing, INT8 Q/K and FP8 V quantization) +
+sage_attn_fwd over one batch of the long-video workload (B=1, H=32, N=55296,
+D=128, BF16 NHD; synthetic, seeded), the largest single-GPU configuration.
+Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload action_dit|mid_video|long_video|ragged|tiny]
                     [--q-gran block64|token|segment64] [--k-gran block64|token|segment64]
+                    [--quant fused|separate] [--normrope] [--op attention|fp8_linear]
 
 value      = attention ops (4*B*H*N^2*D, INT8 QK^T + FP8 PV) per step, all ranks,
              / device time of the whole step (quant + attention), in TOPS;
@@ -22,6 +24,9 @@ e2e        = the same metric through the Python API with pinned host inputs:
              serial figure is reported beside it.
 roofline   = the attention kernel alone: ops / its mean event-timed duration,
              against the INT8/FP8 dense peak derived from the measured BF16 peak.
+workloads  = (default run, one GPU) the other large workloads, eager: attention
+             time, TOPS and roofline fraction, and the GB/s of the fused
+             quantization call and of sage_quant_qk and sage_quant_v standalone.
 cpu_baseline (N=1, rank 0) = the CPU oracle timed on a bounded sample.
 --impl reference runs the CPU oracle (the reference arm) instead.
 Multi-GPU: one process per GPU (torchrun); every rank runs its own batch
@@ -47,6 +52,7 @@ import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 4.5 / 2.25  # nominal dense INT8/FP8 : BF16 tensor throughput ratio
+DEFAULT_WORKLOAD = "long_video"  # the largest single-GPU workload
 
 
 def load_peaks():
@@ -59,43 +65,25 @@ def load_peaks():
 
 
 def kernel_traffic(key: str, sources, workload: str):
-    """DRAM bytes per launch of a kernel from the last ncu capture of it, if that
-    capture was taken on this workload and on the current kernel source
-    (SHA-256 of `sources`); None otherwise."""
+    """DRAM bytes per launch of a kernel from the last ncu capture of it
+    (profiles/ncu_counters.json), if that capture was taken on this workload
+    and on the current kernel source (SHA-256 of `sources`); None otherwise."""
     import hashlib
-    pkg = os.path.join(ROOT, "action_diffusion_transformers_b200")
     try:
-        with open(os.path.join(pkg, "ncu_counters.json")) as f:
+        with open(os.path.join(ROOT, "profiles", "ncu_counters.json")) as f:
             rec = json.load(f)[key]
     except (OSError, KeyError, ValueError):
         return None
     h = hashlib.sha256()
     for name in sources:
-        with open(os.path.join(pkg, "csrc", name), "rb") as f:
+        with open(os.path.join(ROOT, "action_diffusion_transformers_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
         return None
     return rec.get("dram_bytes_per_launch")
 
 
-def attn_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from the last ncu capture,
-    if that capture was taken on this workload and on the current kernel source
-    (SHA-256 of the kernel files); None otherwise."""
-    import hashlib
-    pkg = os.path.join(ROOT, "action_diffusion_transformers_b200")
-    try:
-        with open(os.path.join(pkg, "ncu_counters.json")) as f:
-            rec = json.load(f)["sage_attn_kernel<128, false>"]
-    except (OSError, KeyError, ValueError):
-        return None
-    h = hashlib.sha256()
-    for name in ("sage_attn.cuh", "sage_ptx.cuh"):
-        with open(os.path.join(pkg, "csrc", name), "rb") as f:
-            h.update(f.read())
-    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
-        return None
-    return rec.get("dram_bytes_per_launch")
+ATTN_SOURCES = ("sage_attn.cuh", "sage_ptx.cuh")
 
 
 def parse():
@@ -104,7 +92,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="action_dit", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(synth.WORKLOADS),
+                    help=f"default: {DEFAULT_WORKLOAD}, followed by a summary of the other large workloads")
+    ap.add_argument("--no-summary", action="store_true",
+                    help="skip the per-workload summary that the default run appends")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-gran", default="block64", choices=["block64", "token", "segment64"],
                     help="INT8 scale groups of Q (default: 64-token blocks)")
@@ -570,6 +561,138 @@ def run_fp8_linear(args, rank, world, local):
 
 
 # ----------------------------------------------------------------------------- ours
+SUMMARY_WORKLOADS = ("mid_video", "ragged", "action_dit")
+
+
+class AttnCase:
+    """Device inputs, buffers and the step's calls for one workload."""
+
+    def __init__(self, torch, adt, w, args, stream, qb, kb, vb, nr_host=None):
+        as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
+        self.torch, self.adt, self.w, self.stream = torch, adt, w, stream
+        self.q, self.k, self.v = as_dev(qb), as_dev(kb), as_dev(vb)
+        self.nr = None
+        if nr_host is not None:
+            self.nr = dict(q_w=as_dev(nr_host["q_w"]), k_w=as_dev(nr_host["k_w"]), eps=nr_host["eps"],
+                           cos=torch.from_numpy(nr_host["cos"]).cuda(), sin=torch.from_numpy(nr_host["sin"]).cuda())
+        self.grans = (args.q_gran, args.k_gran)
+        self.buf = self.new_buffers()
+        self.fused = args.quant == "fused" and self.nr is None
+
+    def new_buffers(self):
+        w = self.w
+        return self.adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=self.grans[0],
+                                k_gran=self.grans[1])
+
+    def quant_qk(self, q=None, k=None, buf=None, st=None):
+        q, k, buf, st = q if q is not None else self.q, k if k is not None else self.k, buf or self.buf, st or self.stream
+        if self.nr is None:
+            self.adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                                   buf.workspace, st)
+        else:
+            nr = self.nr
+            self.adt.sage_quant_qk_normrope(q, k, buf.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
+                                            buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
+                                            buf.workspace, st)
+
+    def quant_v(self, v=None, buf=None, st=None):
+        v, buf = v if v is not None else self.v, buf or self.buf
+        self.adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or self.stream)
+
+    def quant_qkv(self, q=None, k=None, v=None, buf=None, st=None):
+        q, k, v = (x if x is not None else d for x, d in ((q, self.q), (k, self.k), (v, self.v)))
+        buf = buf or self.buf
+        self.adt.sage_quant_qkv(q, k, v, buf.shape, 0, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale,
+                                buf.k_mean, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or self.stream)
+
+    def quant_all(self, q=None, k=None, v=None, buf=None, st=None):
+        if self.fused:
+            self.quant_qkv(q, k, v, buf, st)
+        else:
+            self.quant_qk(q, k, buf, st)
+            self.quant_v(v, buf, st)
+
+    def attn(self, buf=None, st=None):
+        buf = buf or self.buf
+        self.adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
+                               buf.v_mean, buf.shape, 0.0, buf.out, False, None, st or self.stream)
+
+    def eager_loop(self, steps, flush, fused):
+        """`steps` eager steps, each after an L2 flush, with events between the
+        launches; returns per-step milliseconds (quant_qk, quant_v or None,
+        quant total, attention, whole step)."""
+        torch, stream = self.torch, self.stream
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            e = ev[i]
+            e[0].record(stream)
+            if fused:
+                self.quant_qkv()
+            else:
+                self.quant_qk()
+                e[1].record(stream)
+                self.quant_v()
+            e[2].record(stream)
+            self.attn()
+            e[3].record(stream)
+        torch.cuda.synchronize()
+        self.adt.sage_check()
+        return dict(qk=None if fused else [e[0].elapsed_time(e[1]) for e in ev],
+                    v=None if fused else [e[1].elapsed_time(e[2]) for e in ev],
+                    quant=[e[0].elapsed_time(e[2]) for e in ev],
+                    attn=[e[2].elapsed_time(e[3]) for e in ev],
+                    step=[e[0].elapsed_time(e[3]) for e in ev])
+
+
+def attn_roofline(w, attn_ms, peaks, src, k_blocks=True):
+    peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    achieved = w.attn_ops / (attn_ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": kernel_traffic(f"sage_attn_kernel<{w.D}, false>", ATTN_SOURCES, w.name) if k_blocks else None,
+            "kernel": f"sage_attn_kernel<{w.D}, {'false' if k_blocks else 'true'}>",
+            "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"}
+
+
+def workload_summary(torch, adt, name, args, stream, flush, peaks, src, gpu):
+    """Eager per-kernel figures of another workload, on one GPU: the fused
+    quantization call and attention (the step), then sage_quant_qk and
+    sage_quant_v as standalone calls (their own GB/s)."""
+    w = synth.WORKLOADS[name]
+    qb, kb, vb = synth.generate(w)
+    case = AttnCase(torch, adt, w, argparse.Namespace(q_gran="block64", k_gran="block64", quant="fused"),
+                    stream, qb, kb, vb)
+    del qb, kb, vb
+    steps = max(3, min(args.steps, 10))
+    for _ in range(3):
+        case.quant_qkv(); case.attn(); case.quant_qk(); case.quant_v()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu)
+    fused = case.eager_loop(steps, flush, True)
+    sep = case.eager_loop(steps, flush, False)
+    clocks = sampler.stop()
+    qk_bytes, v_bytes = quant_bytes(w)
+    mean = statistics.mean
+    attn_ms = mean(fused["attn"] + sep["attn"])
+    roof = attn_roofline(w, attn_ms, peaks, src)
+    out = {"B": w.B, "N": w.N, "H": w.H, "D": w.D, "steps": steps,
+           "step_tops_eager": w.attn_ops * steps / (sum(fused["step"]) / 1e3) / 1e12,
+           "attn_us": 1e3 * attn_ms, "attn_tops": roof["achieved"], "attn_frac": roof["frac"],
+           "attn_traffic": roof["traffic"],
+           "quant_qkv_us": 1e3 * mean(fused["quant"]),
+           "quant_qkv_gbs": (qk_bytes + v_bytes) / (mean(fused["quant"]) / 1e3) / 1e9,
+           "quant_qk_us": 1e3 * mean(sep["qk"]), "quant_qk_gbs": qk_bytes / (mean(sep["qk"]) / 1e3) / 1e9,
+           "quant_v_us": 1e3 * mean(sep["v"]), "quant_v_gbs": v_bytes / (mean(sep["v"]) / 1e3) / 1e9,
+           "hbm_frac": {k: v / peaks["hbm_gbs"] for k, v in (
+               ("quant_qkv", (qk_bytes + v_bytes) / (mean(fused["quant"]) / 1e3) / 1e9),
+               ("quant_qk", qk_bytes / (mean(sep["qk"]) / 1e3) / 1e9),
+               ("quant_v", v_bytes / (mean(sep["v"]) / 1e3) / 1e9))},
+           "clocks": clocks}
+    del case
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     rank, world, local = rank_env()
@@ -577,6 +700,9 @@ def main():
         if rank == 0:
             print(json.dumps({"peaks": measure_peaks(), "shape": "8192^3", "best_of": 20}), flush=True)
         return
+    summary = args.workload is None and args.op == "attention" and not args.no_summary
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD if args.op == "attention" else "action_dit"
     if args.impl == "reference":
         run_reference(args, rank)
         return
@@ -590,7 +716,7 @@ def main():
 
     torch.cuda.set_device(local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     if args.op == "fp8_linear":
         run_fp8_linear(args, rank, world, local)
@@ -601,78 +727,29 @@ def main():
     if args.normrope:
         qb, kb = synth.projection_outputs(w)
         nr_host = synth.normrope_inputs(w)
-    as_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
-    q, k, v = as_dev(qb), as_dev(kb), as_dev(vb)
-    nr = None
-    if nr_host is not None:
-        nr = dict(q_w=as_dev(nr_host["q_w"]), k_w=as_dev(nr_host["k_w"]), eps=nr_host["eps"],
-                  cos=torch.from_numpy(nr_host["cos"]).cuda(), sin=torch.from_numpy(nr_host["sin"]).cuda())
-    buf = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=args.q_gran, k_gran=args.k_gran)
     stream = torch.cuda.current_stream()
+    case = AttnCase(torch, adt, w, args, stream, qb, kb, vb, nr_host)
+    q, k, v, buf, nr, fused = case.q, case.k, case.v, case.buf, case.nr, case.fused
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-
-    def quant_qk(q=q, k=k, buf=buf, st=None):
-        st = st or stream
-        if nr is None:
-            adt.sage_quant_qk(q, k, buf.shape, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                              buf.workspace, st)
-        else:
-            adt.sage_quant_qk_normrope(q, k, buf.shape, nr["q_w"], nr["k_w"], nr["cos"], nr["sin"], nr["eps"],
-                                       buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                                       buf.workspace, st)
-
-    def quant_v(v=v, buf=buf, st=None):
-        adt.sage_quant_v(v, buf.shape, buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or stream)
-
-    fused = args.quant == "fused" and nr is None
-
-    def quant_qkv(q=q, k=k, v=v, buf=buf, st=None):
-        adt.sage_quant_qkv(q, k, v, buf.shape, 0, buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.k_mean,
-                           buf.v_codes_t, buf.v_scale, buf.v_mean, buf.workspace, st or stream)
-
-    def quant_all(q=q, k=k, v=v, buf=buf, st=None):
-        if fused:
-            quant_qkv(q, k, v, buf, st)
-        else:
-            quant_qk(q, k, buf, st)
-            quant_v(v, buf, st)
-
-    def attn(buf=buf, st=None):
-        adt.sage_attn_fwd(buf.q_codes, buf.q_scale, buf.k_codes, buf.k_scale, buf.v_codes_t, buf.v_scale,
-                          buf.v_mean, buf.shape, 0.0, buf.out, False, None, st or stream)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     for _ in range(max(3, args.warmup)):
-        quant_all(); attn()
+        case.quant_all(); case.attn()
     adt.sage_check()
     torch.cuda.synchronize()
     barrier()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    sampler = ClockSampler(gpu_id_for(local))
+    gpu = gpu_id_for(local)
+    sampler = ClockSampler(gpu)
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    for i in range(K):
-        flush.fill_(i & 0xFF)
-        e = ev[i]
-        e[0].record(stream)
-        if fused:
-            quant_qkv()
-        else:
-            quant_qk()
-            e[1].record(stream)
-            quant_v()
-        e[2].record(stream)
-        attn()
-        e[3].record(stream)
-    torch.cuda.synchronize()
+    eager = case.eager_loop(K, flush, fused)
     barrier()
-    adt.sage_check()
     eager_out = buf.out.clone()
 
     # The same launches captured once into a CUDA graph and replayed: the
@@ -682,8 +759,8 @@ def main():
     side.wait_stream(stream)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=side):
-        quant_all(st=side)
-        attn(st=side)
+        case.quant_all(st=side)
+        case.attn(st=side)
     torch.cuda.synchronize()
     graph.replay()
     torch.cuda.synchronize()
@@ -700,14 +777,10 @@ def main():
     adt.sage_check()
     if not torch.equal(buf.out, eager_out):
         raise RuntimeError("the graph replay's output differs from the eager step's")
+    del graph, eager_out
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in ev]
-    quant_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    qk_ms = None if fused else [e[0].elapsed_time(e[1]) for e in ev]
-    v_ms = None if fused else [e[1].elapsed_time(e[2]) for e in ev]
-    at_ms = [e[2].elapsed_time(e[3]) for e in ev]
     ops = w.attn_ops
-    eager_value = job_tops(world, ops, K, max_over_ranks(sum(step_ms), world, "cuda"))
+    eager_value = job_tops(world, ops, K, max_over_ranks(sum(eager["step"]), world, "cuda"))
     max_total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev), world, "cuda")
     value = job_tops(world, ops, K, max_total_ms)
 
@@ -719,11 +792,13 @@ def main():
     # while step i computes; events order each slot's reuse.
     pin = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()  # noqa: E731
     hq, hk, hv = pin(qb), pin(kb), pin(vb)
+    h2d = 3 * qb.nbytes
+    del qb, kb, vb
     hout = [torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory() for _ in range(2)]
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for _ in range(2):
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        quant_all(); attn()
+        case.quant_all(); case.attn()
         hout[0].copy_(buf.out, non_blocking=True)
     torch.cuda.synchronize()
     barrier()
@@ -731,7 +806,7 @@ def main():
         flush.fill_(i & 0xFF)
         e2e_ev[i][0].record(stream)
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True); v.copy_(hv, non_blocking=True)
-        quant_all(); attn()
+        case.quant_all(); case.attn()
         hout[0].copy_(buf.out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
@@ -739,7 +814,7 @@ def main():
     adt.sage_check()
     e2e_serial = job_tops(world, ops, K, max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), world, "cuda"))
 
-    buf2 = adt.Buffers(w.B, w.N, w.H, w.D, cu_seqlens=w.cu_seqlens, q_gran=args.q_gran, k_gran=args.k_gran)
+    buf2 = case.new_buffers()
     slots = [(q, k, v, buf), (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), buf2)]
 
     def copy_in(j):
@@ -747,8 +822,8 @@ def main():
             d.copy_(h, non_blocking=True)
 
     def compute(j):
-        quant_all(*slots[j])
-        attn(slots[j][3])
+        case.quant_all(*slots[j])
+        case.attn(slots[j][3])
 
     def copy_out(j):
         hout[j].copy_(slots[j][3].out, non_blocking=True)
@@ -762,36 +837,44 @@ def main():
     out_ok = torch.equal(hout[(K - 1) & 1], buf2.out.cpu() if (K - 1) & 1 else buf.out.cpu())
     if not out_ok:
         raise RuntimeError("pipelined e2e: the copied-out output differs from the device result")
-    h2d = 3 * qb.nbytes
     d2h = buf.out.numel() * buf.out.element_size()
+    del slots, buf2, hout
 
     # --------------------------------------------------------------- roofline, baseline
     peaks, src = load_peaks()
-    peak = peaks["bf16_tflops"] * INT8_PER_BF16
     k_blocks = args.k_gran == "block64"
-    attn_mean_ms = statistics.mean(at_ms)
-    achieved = ops / (attn_mean_ms / 1e3) / 1e12
+    attn_mean_ms = statistics.mean(eager["attn"])
+    roofline = attn_roofline(w, attn_mean_ms, peaks, src, k_blocks)
     qk_bytes, v_bytes = quant_bytes(w, args.q_gran, args.k_gran)
     if nr is not None:
         qk_bytes += w.N * w.D // 2 * 8 + 2 * w.D * 2          # cos / sin tables once, the two weights
+    mean = statistics.mean
     if fused:
-        quant_us = {"quant_qkv": 1e3 * statistics.mean(quant_ms), "attn": 1e3 * attn_mean_ms}
-        quant_gbs = {"quant_qkv": (qk_bytes + v_bytes) / (statistics.mean(quant_ms) / 1e3) / 1e9,
+        quant_us = {"quant_qkv": 1e3 * mean(eager["quant"]), "attn": 1e3 * attn_mean_ms}
+        quant_gbs = {"quant_qkv": (qk_bytes + v_bytes) / (mean(eager["quant"]) / 1e3) / 1e9,
                      "peak_hbm_gbs": peaks["hbm_gbs"]}
     else:
-        quant_us = {"quant_qk": 1e3 * statistics.mean(qk_ms), "quant_v": 1e3 * statistics.mean(v_ms),
+        quant_us = {"quant_qk": 1e3 * mean(eager["qk"]), "quant_v": 1e3 * mean(eager["v"]),
                     "attn": 1e3 * attn_mean_ms}
-        quant_gbs = {"quant_qk": qk_bytes / (statistics.mean(qk_ms) / 1e3) / 1e9,
-                     "quant_v": v_bytes / (statistics.mean(v_ms) / 1e3) / 1e9, "peak_hbm_gbs": peaks["hbm_gbs"]}
+        quant_gbs = {"quant_qk": qk_bytes / (mean(eager["qk"]) / 1e3) / 1e9,
+                     "quant_v": v_bytes / (mean(eager["v"]) / 1e3) / 1e9, "peak_hbm_gbs": peaks["hbm_gbs"]}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # about 10-30 s of CPU work on the host: 4 heads, 2^26 (query row, key) pairs
         heads = min(4, w.H)
         rows = max(1, min(w.N, (1 << 26) // (heads * w.N)))
-        o_ops, o_dt = oracle_sample(w, qb, kb, vb, rows, heads, args.q_gran, args.k_gran, nr_host)
+        hb = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+        o_ops, o_dt = oracle_sample(w, hb(hq), hb(hk), hb(hv), rows, heads, args.q_gran, args.k_gran, nr_host)
         cpu = {"value": o_ops / o_dt / 1e12, "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+               "cores_note": "BLAS threads of the score products; the oracle's other steps run on one core",
                "sample": f"{heads} heads of batch 0: full K/V quantization of those heads + attention for "
                          f"{rows} query rows each ({o_dt:.1f} s)"}
+    del case, q, k, v, buf, hq, hk, hv
+    torch.cuda.empty_cache()
+    others = None
+    if summary and rank == 0 and world == 1:
+        others = {name: workload_summary(torch, adt, name, args, stream, flush, peaks, src, gpu)
+                  for name in SUMMARY_WORKLOADS if name != w.name}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -805,11 +888,10 @@ def main():
                    "seq_len": w.N, "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write)",
                    "q_gran": args.q_gran, "k_gran": args.k_gran,
                    "qk_prologue": "rmsnorm+rope" if nr is not None else None},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": attn_traffic(w.name) if k_blocks else None,
-                     "kernel": f"sage_attn_kernel<{w.D}, {'false' if k_blocks else 'true'}>",
-                     "peak_source": f"{src} bf16 burst {peaks['bf16_tflops']} x {INT8_PER_BF16} (int8/fp8 dense)"},
+        "roofline": roofline,
         "kernels_us": quant_us,
+        "kernels_us_note": "per-kernel means from the eager loop (events between launches); value and "
+                           "ms_per_step from graph replays, which trim the gaps between launches",
         "quant_gbs": quant_gbs,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -820,6 +902,8 @@ def main():
         "eager_value": eager_value,
         "clocks": clocks,
     }
+    if others is not None:
+        line["workloads"] = others
     print(json.dumps(line), flush=True)
 
 

@@ -307,7 +307,10 @@ SAGE_API sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_
  * before any stream capture.  Every call on a device shares the one array and
  * it keeps the last call's contents (nothing in it needs to start at zero):
  * calls that overlap on the GPU (concurrent streams) race on it, so order
- * them on one stream or with events.
+ * them on one stream or with events.  The looked-up address is kept for the
+ * life of the process: do not call this entry point on a device after
+ * cudaDeviceReset() (or anything else that re-creates its primary context),
+ * because the kept address then belongs to the old context.
  */
 #define SAGE_QK_STATIC_SCRATCH_BYTES (8u << 20)
 SAGE_API sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s,
