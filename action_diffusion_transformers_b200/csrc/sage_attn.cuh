@@ -49,7 +49,6 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kSBiasBits = 0x4B400000u;   // S accumulates onto these bits
 constexpr float kSBias = 12582912.0f;          // their float value, 1.5 * 2^23
 constexpr float kLog2P8 = 8.8073549220576041f; // log2(448): the P scale, folded into the exponent
-constexpr float kMaxSlack = 2.0f;                // a raised running max sits this far above the tile max
 
 template <int D>
 struct AttnSmem {
@@ -337,9 +336,8 @@ struct SoftmaxTile {
       smin0 = fminf(mn[0], mn[1]);       // biased
       smin1 = fminf(mn[2], mn[3]);
     }
-    // A raised running max sits kMaxSlack above the tile max, so that later
-    // tiles rarely move it (and alpha is exactly 1 while it stays).
-    const float m_new = tmax > m ? __fadd_rn(tmax, kMaxSlack) : m;
+    // Running row max (alpha is exactly 1 while it stays).
+    const float m_new = fmaxf(m, tmax);
     const float alpha = exp2_fixed5(__fsub_rn(m, m_new));
     const float e = __fsub_rn(kLog2P8, m_new);
     const float off0 = __fmaf_rn(-kSBias, c0, e);

@@ -225,7 +225,7 @@ SAGE_API sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_
  * Per 128-row query tile and 128-key tile: S = Qc Kc^T exactly in INT32 on the
  * tensor cores; t = RN(S * c) with c = RN(RN(qs_i * ks_j) * RN(sm_scale *
  * log2 e)), qs_i / ks_j the scales of the groups holding query i / key j;
- * running row max m, set to RN(max t + 2) when a tile's max exceeds it;
+ * running row max m = max(m, max t);
  * y = exp2(RN((S + B) * c + e')) with B = 1.5 * 2^23, e = RN(log2 448 - m)
  * and e' = RN(e - B * c), exp2 a fixed binary32 algorithm (Cody-Waite split,
  * quadratic, exponent-field add); l accumulates y; P8 = E4M3(y) (<= 448);

@@ -31,8 +31,9 @@ against brute-force FP64 softmax attention; smoothing by the softmax shift
 invariance; closed forms for degenerate inputs; the softmax exp2 against
 numpy's exp2 within its stated error bound and exactly at integers; the fused
 multiply-add against exact rational rounding; the exponent formed on biased
-scores against exact rationals; the running-max slack by its rule and, with
-the score bias, by brute-force softmax).  With the exp2 and the FMA
+scores against exact rationals and, with the score bias, by brute-force
+softmax; the contract's softmax against a plain reading of it, attn_fwd_plain,
+within a bound derived from the E4M3 step of P).  With the exp2 and the FMA
 fixed by the contract, the E4M3 codes of P are reproducible; attention parity
 keeps a tolerance for the tensor core's FP32 summation order and the order of
 the row-sum additions.
@@ -56,7 +57,6 @@ E4M3_MAX = 448.0
 LOG2E = 1.4426950408889634
 LOG2_P_UNIT = np.float32(math.log2(E4M3_MAX))   # RN32(log2 448), the P scale in the exponent
 S_BIAS = np.float32(12582912.0)  # 1.5 * 2^23: integer scores are carried as the binary32 S + S_BIAS
-MAX_SLACK = np.float32(2.0)      # a raised running max is set this far (exp2 units) above the tile max
 
 
 def npad(n: int) -> int:
@@ -337,7 +337,7 @@ def _identity(x):
 
 
 def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2_alpha, quant_p,
-                 log2_p_unit, two_pass=False, s_bias=0.0, slack=0.0):
+                 log2_p_unit, two_pass=False, s_bias=0.0):
     """Online-softmax attention over 128-key tiles for one (b, h).
 
     S         [R, >= n_keys] float64: exact score numerators (INT32 dot
@@ -357,25 +357,21 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
     s_bias    the bias B the scores are carried on (S_BIAS with quantization
               on: the integer S as the binary32 S + B, exact for |S| < 2^22;
               0 with it off).
-    slack     how far above the tile max a raised running max is set (MAX_SLACK
-              with quantization on, 0 with it off).
 
     Per tile j (keys j0..j1-1, those >= n_keys excluded):
       t     = rn(S * c)                          scores in the exp2 domain
-      m_new = rn(max_k t + slack) if max_k t > m else m
-                                                 running row max, an upper bound
-                                                 of every t so far
+      m_new = max(m, max_k t)                    running row max
       alpha = exp2_alpha(rn(m - m_new))          (0 on the first tile, m = -inf;
                                                  exactly 1 while m is unchanged)
       e     = rn(log2_p_unit - m_new)
       e'    = fma(-B, c, e)                      the exponent offset for biased scores
-      y     = exp2(fma(S + B, c, e'))            = P~ * 448 * 2^-(m_new - max t),
-                                                 P~ = exp2(t - m_new) up to e's rounding
+      y     = exp2(fma(S + B, c, e'))            = P~ * 448, P~ = exp2(t - m_new)
+                                                 up to e's rounding
       l     = rn(rn(l * alpha) + rn(sum_k y))    row sum of the unquantized y
       P8    = quant_p(y)                         E4M3 code of y (<= 448)
       acc   = rn(rn(acc * alpha) + rn(P8 @ V))   product sum exact, then rounded
     Epilogue: o = fma(rn(acc * out_mult), rn(1 / l), out_add); the P scale
-    and the slack cancel between acc and l.
+    cancels between acc and l.
     With B = 0, e' = e and y = exp2(fma(S, c, e)); with B != 0 the single
     rounding of e' shifts every exponent of a (row, c) pair by the same
     amount, at most half an ulp of B * c (below 1.5 c, under two units of the
@@ -399,7 +395,7 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
         c = col_mult(j0, j1)
         t = rn(S[:, j0:j1] * c)
         tmax = t.max(axis=1)
-        m_new = m if two_pass else np.where(tmax > m, rn(tmax + np.float64(slack)), m)
+        m_new = m if two_pass else np.maximum(m, tmax)
         with np.errstate(invalid="ignore"):
             alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2_alpha(rn(m - m_new)), dtype=np.float64))
         if two_pass:
@@ -445,7 +441,7 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     the scales of the groups that hold token i of Q and token j of K:
         c = RN32(RN32(qs[i] * ks[j]) * RN32(sm_scale * log2 e)),
     the P scale 448 enters the exponent as RN32(log2 448) (P8 = E4M3(y), y =
-    P~ * 448 below the slack of the running max, with the exponent formed by
+    P~ * 448 with P~ = exp2(t - m) <= 1, with the exponent formed by
     one fused multiply-add on the biased score S + S_BIAS), the row sum holds y
     and the output factor is the V scale itself.
     sm_scale None or <= 0 means 1/sqrt(D).
@@ -478,21 +474,123 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
         o, m, l = _attend_rows(S, col_mult, Vt, v_scale[b, h].astype(np.float64),
                                v_mean[b, h].astype(np.float64), N, rn32, fma32, exp2_contract,
                                _exp2_alpha, _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass,
-                               s_bias=S_BIAS, slack=MAX_SLACK)
+                               s_bias=S_BIAS)
         out[b, :, h, :] = o
         lse[b, h] = rn32((m + np.log2(l) - math.log2(E4M3_MAX)) * math.log(2.0))
     return (out, lse) if want_lse else out
 
 
+# ----------------------------------------------------------------------------
+# The plain reading of the FP32 online softmax, kept beside the contract
+# ----------------------------------------------------------------------------
+def _attend_rows_plain(S, col_mult, Vt, out_mult, out_add, n_keys, rn, exp2, quant_p):
+    """Online softmax over 128-key tiles in its plainest FP32 reading.
+
+    The pages fix INT8 QK, FP8 PV, FP32 accumulation and an FP32 online
+    softmax ("FLUX.3 Action RTX 5090 report", 02 ENGINEERING, card 03;
+    "MiniMax H3 on DGX Spark", 01 Precision map) and nothing finer.  This
+    variant takes every step as written there, with no choice made for speed:
+    exp2 evaluated in FP64 and rounded once, no score bias, the running max
+    exactly the largest score so far, P~ in [0, 1] scaled by 448 only for its
+    E4M3 code, and l summed from the unquantized P~.
+
+    S, col_mult, Vt, out_mult, out_add, n_keys as in _attend_rows; rn the
+    rounding after every step (rn32, or identity), exp2 the exponential
+    (RN32 of the FP64 exp2, or np.exp2), quant_p the P quantizer applied to
+    448 * P~ (E4M3 round trip, or identity).  Per tile j:
+      t     = rn(S * c)
+      m_new = max(m, max_k t)
+      alpha = exp2(rn(m - m_new))                (0 on the first tile)
+      P~    = exp2(rn(t - m_new))                in [0, 1]
+      l     = rn(rn(l * alpha) + rn(sum_k P~))
+      acc   = rn(rn(acc * alpha) + rn(quant_p(rn(448 * P~)) @ V))
+    Epilogue: o = rn(acc * out_mult / (448 * l) + out_add), in FP64 then
+    rounded once.  Returns (o [R, D], m [R], l [R]).
+    """
+    R = S.shape[0]
+    D = Vt.shape[0]
+    nkv = (n_keys + TILE - 1) // TILE
+    m = np.full(R, -np.inf)
+    l = np.zeros(R)
+    acc = np.zeros((R, D))
+    for j in range(nkv):
+        j0, j1 = j * TILE, min(n_keys, (j + 1) * TILE)
+        t = rn(S[:, j0:j1] * col_mult(j0, j1))
+        m_new = np.maximum(m, t.max(axis=1))
+        with np.errstate(invalid="ignore"):
+            alpha = np.where(np.isneginf(m), 0.0, np.asarray(exp2(rn(m - m_new)), dtype=np.float64))
+        p = np.asarray(exp2(rn(t - m_new[:, None])), dtype=np.float64)
+        l = rn(rn(l * alpha) + rn(p.sum(axis=1)))
+        p8 = np.asarray(quant_p(rn(np.float64(E4M3_MAX) * p)), dtype=np.float64)
+        acc = rn(rn(acc * alpha[:, None]) + rn(p8 @ Vt[:, j0:j1].T))
+        m = m_new
+    o = rn(acc * out_mult[None, :] / (np.float64(E4M3_MAX) * l)[:, None] + out_add[None, :])
+    return np.asarray(o, dtype=np.float64), m, l
+
+
+def _exp2_rn32(x):
+    """exp2 in FP64, rounded once to binary32."""
+    return rn32(np.exp2(np.asarray(x, dtype=np.float64)))
+
+
+def attn_fwd_plain(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
+                   sm_scale=None, rows=None, heads=None, quantize_p=True):
+    """A6-A10 on the same quantized operands as attn_fwd, with the softmax in
+    its plain reading (_attend_rows_plain): the yardstick that the contract's
+    exponent (fixed quadratic exp2, biased score) is bounded against.  The
+    score multiplier c, the E4M3 codes of V and the V-mean add-back are
+    attn_fwd's.  quantize_p=False keeps 448 * P~ unquantized in the PV product
+    (its distance from the quantized result is the plain reading's own P
+    quantization error).  Returns float32 [B, R, H, D]."""
+    B, H, Np, D = q_codes.shape
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = default_sm_scale(D)
+    sl2e = exp2_scale(sm_scale)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, rows.shape[0], H, D), dtype=np.float32)
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in heads:
+        S = q_codes[b, h, rows].astype(np.float64) @ k_codes[b, h, :N].astype(np.float64).T
+        qs = token_scales(q_scale[b, h], Np)[rows]
+        ks = token_scales(k_scale[b, h], Np)
+
+        def col_mult(j0, j1, qs=qs, ks=ks):
+            return rn32(rn32(qs[:, None].astype(np.float64) * ks[None, j0:j1]) * np.float64(sl2e))
+
+        o, _, _ = _attend_rows_plain(S, col_mult, e4m3_decode(v_codes_t[b, h, :, :N]),
+                                     v_scale[b, h].astype(np.float64), v_mean[b, h].astype(np.float64), N,
+                                     rn32, _exp2_rn32, _e4m3_round_trip if quantize_p else _identity)
+        out[b, :, h, :] = o
+    return out
+
+
+def attn_plain_unquantized(q, k, v, N, sm_scale=None, rows=None, heads=None):
+    """_attend_rows_plain with quantization and rounding OFF, all in FP64 (no
+    smoothing): pins the plain tile loop against brute-force softmax
+    attention.  q, k, v float64 [B, N, H, D]; returns float64 [B, R, H, D]."""
+    B, _, H, D = q.shape
+    if sm_scale is None or sm_scale <= 0:
+        sm_scale = 1.0 / math.sqrt(D)
+    c = sm_scale * LOG2E
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    out = np.zeros((B, rows.shape[0], H, D))
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
+    for b, h in heads:
+        S = q[b, rows, h, :] @ k[b, :N, h, :].T
+        o, _, _ = _attend_rows_plain(S, lambda j0, j1: c, v[b, :N, h, :].T, np.ones(D), np.zeros(D), N,
+                                     _identity, np.exp2, _identity)
+        out[b, :, h, :] = o
+    return out
+
+
 def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
-                     smooth_v=True, heads=None, s_bias=0.0, slack=0.0):
+                     smooth_v=True, heads=None, s_bias=0.0):
     """The same tile loop with quantization OFF, all in FP64.
 
     q, k, v: float64 [B, N, H, D].  Scores are exact FP64 dot products, the
     multiplier is sm_scale * log2 e, P is not quantized (p_unit 1), V is
     centred by its FP64 mean (smooth_v) and K by its FP64 mean (smooth_k).
-    s_bias, slack: the score bias and the running-max slack of the quantized
-    loop, which must cancel.  Used to pin the tile loop, the rescaling, the
+    s_bias: the score bias of the quantized loop, which must cancel.  Used to pin the tile loop, the rescaling, the
     biased exponent and the smoothing algebra against brute-force softmax
     attention.  Returns float64 [B, R, H, D].
     """
@@ -513,7 +611,7 @@ def attn_unquantized(q, k, v, N, sm_scale=None, rows=None, smooth_k=True,
         S = Q @ K.T
         o, _, _ = _attend_rows(S, lambda j0, j1: c, (V - mean).T, np.ones(D), mean,
                                N, _identity, _fma_exact, np.exp2, np.exp2, _identity, 0.0,
-                               s_bias=s_bias, slack=slack)
+                               s_bias=s_bias)
         out[b, :, h, :] = o
     return out
 
@@ -538,11 +636,16 @@ def attn_exact_fp64(q, k, v, N, sm_scale=None, rows=None, heads=None):
 
 
 def sage_pipeline(q_bits, k_bits, v_bits, sm_scale=None, rows=None, heads=None,
-                  two_pass=False, q_gran="block64", k_gran="block64", cu_seqlens=None):
-    """Whole path A1-A10 from BF16 inputs: returns (fp32 output, intermediates)."""
+                  two_pass=False, q_gran="block64", k_gran="block64", cu_seqlens=None, plain=False):
+    """Whole path A1-A10 from BF16 inputs: returns (fp32 output, intermediates).
+    plain: the softmax in its plain reading (attn_fwd_plain) instead of the contract."""
     N = q_bits.shape[1]
     qk = quant_qk(q_bits, k_bits, q_gran, k_gran, cu_seqlens)
     vv = quant_v(v_bits)
+    if plain:
+        o = attn_fwd_plain(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"], vv["v_codes_t"],
+                           vv["v_scale"], vv["v_mean"], N, sm_scale=sm_scale, rows=rows, heads=heads)
+        return o, dict(qk, **vv)
     o = attn_fwd(qk["q_codes"], qk["q_scale"], qk["k_codes"], qk["k_scale"],
                  vv["v_codes_t"], vv["v_scale"], vv["v_mean"], N, sm_scale=sm_scale,
                  rows=rows, heads=heads, two_pass=two_pass)

@@ -8,8 +8,15 @@ the oracle computes head by head and row by row:
   max-abs <= 2e-3 and cosine >= 0.9999 against the oracle, and cosine against
   exact FP64 attention on the BF16 inputs >= 0.999 -- except on the
   long-video workload, whose Student-t(3) rows make a few softmax rows hinge
-  on large INT8 scores: there the method itself (the oracle, and equally a
-  per-token INT8 variant) reaches about 0.998, so the check is >= 0.997;
+  on large INT8 scores.  There the accuracy target of 0.999 against exact
+  FP64 is NOT met: the method reaches about 0.998 whichever softmax is used
+  (the contract, the plain reading, a per-token INT8 variant alike; with
+  exact Q/K it is 0.9996), so this check only guards against a regression
+  (>= 0.997);
+* the FP32 output against the plain reading of the softmax (oracle
+  attn_fwd_plain: exp2 in FP64, no score bias, l from the unquantized P~):
+  cosine >= 0.9999 and max-abs <= 2e-2, the bound the contract itself keeps
+  from that reading (tests/test_contract_vs_plain.py);
 * the BF16 output equals the RNE rounding of the FP32 output on those rows;
 * the LSE of those rows within 1e-4 (relative to max(1, |lse|)) of the oracle's.
 A D = 64 shape with many KV tiles and a ragged tail runs the same checks, and
@@ -96,6 +103,14 @@ def test_full_size_sampled_parity(adt, name, q_gran, k_gran):
         err = np.abs(g32 - ref).max()
         assert err <= 2e-3, f"{name} head {(b, h)}: max-abs {err}"
         assert _cos(g32, ref) >= 0.9999
+        if q_gran == "block64" and k_gran == "block64":
+            plain = so.attn_fwd_plain(ref_qk["q_codes"], ref_qk["q_scale"], ref_qk["k_codes"], ref_qk["k_scale"],
+                                      ref_v["v_codes_t"], ref_v["v_scale"], ref_v["v_mean"], w.N,
+                                      rows=rows)[0, :, 0, :]
+            d_plain = float(np.abs(g32 - plain).max())
+            print(f"{name} head {(b, h)}: vs plain reading max-abs {d_plain:.3e} cos {_cos(g32, plain):.7f}")
+            assert _cos(g32, plain) >= 0.9999
+            assert d_plain <= 2e-2
         exact = so.attn_exact_fp64(*(synth.bits_to_f64(x[sl]) for x in (qb, kb, vb)), w.N, rows=rows)[0, :, 0, :]
         floor = 0.997 if name == "long_video" else 0.999
         assert _cos(g32, exact) >= floor, f"{name} head {(b, h)}: cos vs exact {_cos(g32, exact)}"

@@ -152,10 +152,7 @@ def _cos(a, b):
 @pytest.mark.parametrize("N,D", [(256, 64), (512, 128)])
 def test_token_q_scales_help_when_some_rows_are_large(N, D):
     # 1 query row in 32 is 20x larger: with 64-token blocks it sets the scale of
-    # its whole block, so the other rows keep only a few INT8 levels.  The
-    # softmax rows of such a case are peaked, so this also bounds how much of a
-    # row's weight the running-max slack may push into E4M3's subnormals (at a
-    # slack of 4 the per-token error on 1x512x2x128 rises from 0.024 to 0.041).
+    # its whole block, so the other rows keep only a few INT8 levels.
     B, H = 1, 2
     q, k, v = synth.generate(synth.custom(B, N, H, D, seed=9, k_sigma=2.0, v_sigma=1.0))
     qf = synth.bits_to_f64(q).astype(np.float32)
