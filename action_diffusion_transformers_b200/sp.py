@@ -12,7 +12,9 @@ all-to-all returns its heads' output rows to the ranks that own the tokens.
 The exchange uses torch.distributed.all_to_all_single (NCCL over NVLink on
 GPUs, gloo on CPU); H and N must be multiples of P.  Chunks are ordered by
 rank, so the gathered token order is the global one and cu_seqlens of the
-joint sequence apply unchanged.
+joint sequence apply unchanged.  Under gloo, device tensors are exchanged
+through host memory (gloo moves host buffers); the attention itself still runs
+in the CUDA kernels on each rank's GPU.
 """
 from __future__ import annotations
 
@@ -28,6 +30,8 @@ def _exchange(send: torch.Tensor, group) -> torch.Tensor:
     """all_to_all_single of a [P, ...] tensor, moved as bytes: 2-byte elements
     (BF16, or their int16 bit patterns) travel as int32 pairs, a type every
     backend carries."""
+    if send.is_cuda and dist.get_backend(group) == "gloo":
+        return _exchange(send.cpu(), group).to(send.device)
     words = send.view(torch.int32) if send.element_size() == 2 and send.shape[-1] % 2 == 0 else send
     recv = torch.empty_like(words)
     dist.all_to_all_single(recv, words, group=group)
