@@ -71,14 +71,14 @@ def kernel_traffic(key: str, sources, workload: str):
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_counters.json")) as f:
-            rec = json.load(f)[key]
+            rec = json.load(f)[key][workload]
     except (OSError, KeyError, ValueError):
         return None
     h = hashlib.sha256()
     for name in sources:
         with open(os.path.join(ROOT, "action_diffusion_transformers_b200", "csrc", name), "rb") as f:
             h.update(f.read())
-    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
+    if rec.get("source_sha256") != h.hexdigest():
         return None
     return rec.get("dram_bytes_per_launch")
 
