@@ -149,13 +149,15 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
 // Per (b, 64-token block c, channel): s = ((0 + x_{64c}) + x_{64c+1}) + ... in
 // token order, in FP64.  Grid (nsb, B, ceil(HD / (8*blockDim))).
 // ----------------------------------------------------------------------------
+// tx: the thread's index in its group of 128 (threadIdx.x for a 128-thread CTA).
 template <bool kMinMax>
 __device__ __forceinline__ void colstats_body(int bx, int by, int bz, const uint16_t* __restrict__ x, int N,
                                               int HD, int64_t tok_stride, int nsb, double* __restrict__ psum,
-                                              float* __restrict__ pmin, float* __restrict__ pmax) {
+                                              float* __restrict__ pmin, float* __restrict__ pmax,
+                                              int tx = static_cast<int>(threadIdx.x)) {
   const int c = bx;
   const int b = by;
-  const int ch0 = (bz * 128 + threadIdx.x) * 8;
+  const int ch0 = (bz * 128 + tx) * 8;
   if (ch0 >= HD) return;
   const int n0 = c * kSumBlock;
   const int n1 = min(N, n0 + kSumBlock);
@@ -470,10 +472,12 @@ __device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint
       if (n < N) {
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
-          const __nv_bfloat162 c2 =
-              __floats2bfloat162_rn(__fsub_rn(x[t][i], mean[i]), __fsub_rn(x[t][i + 1], mean[i + 1]));
-          x[t][i] = __low2float(c2);
-          x[t][i + 1] = __high2float(c2);
+          const f32x2_t dv = x2_sub(x2_pack(__float_as_uint(x[t][i]), __float_as_uint(x[t][i + 1])),
+                                    x2_pack(__float_as_uint(mean[i]), __float_as_uint(mean[i + 1])));
+          const __nv_bfloat162 c2 = __floats2bfloat162_rn(x2_lo(dv), x2_hi(dv));
+          const uint32_t cb = *reinterpret_cast<const uint32_t*>(&c2);
+          x[t][i] = __uint_as_float(cb << 16);
+          x[t][i + 1] = __uint_as_float(cb & 0xFFFF0000u);
         }
       }  // padded rows stay 0
     }
@@ -505,18 +509,23 @@ __device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint
   }
   const int64_t bh = static_cast<int64_t>(b) * H + h;
   int8_t* dst = is_k ? k_codes : q_codes;
+  // code = RNE(RN(x * inv)) in [-127, 127] without a clamp: |x| <= amax gives
+  // |x * inv| <= 127 * (1 + 2^-24), which rounds to at most 127.  After the
+  // 1.5 * 2^23 addition the integer sits in the low bits of the float, so the
+  // low byte of each word is the code's two's-complement byte; three byte
+  // permutes gather four of them.  The product and the addition are the
+  // scalar rounding intrinsics, which the compiler never fuses into one FMA
+  // (a fused RN(x * inv + 1.5 * 2^23) would skip the rounding of the product).
 #pragma unroll
   for (int t = 0; t < kTPT; ++t) {
     const int n = tile * kTokens + r0 + t * kRPP;
     const float iv = inv[t / kHalf];
-    uint32_t w[2] = {0u, 0u};
+    uint32_t cw[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int c = rne_small(__fmul_rn(x[t][i], iv));
-      c = max(-127, min(127, c));
-      w[i >> 2] |= (static_cast<uint32_t>(c) & 0xFFu) << (8 * (i & 3));
-    }
-    *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w[0], w[1]);
+    for (int i = 0; i < 8; ++i) cw[i] = __float_as_uint(__fadd_rn(__fmul_rn(x[t][i], iv), 12582912.0f));
+    const uint32_t w0 = __byte_perm(__byte_perm(cw[0], cw[1], 0x0040), __byte_perm(cw[2], cw[3], 0x0040), 0x5410);
+    const uint32_t w1 = __byte_perm(__byte_perm(cw[4], cw[5], 0x0040), __byte_perm(cw[6], cw[7], 0x0040), 0x5410);
+    *reinterpret_cast<uint2*>(dst + (bh * Npad + n) * D + d0) = make_uint2(w0, w1);
   }
   if (threadIdx.x < kSlots)
     (is_k ? k_scale : q_scale)[bh * (Npad / kQKBlock) + tile * kSlots + threadIdx.x] = threadIdx.x == 0 ? scale[0] : scale[1];
