@@ -3,8 +3,9 @@
 // One CTA computes one 128-row query tile of one (b, h).  Warp roles:
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Per tile it
 //              reads its 128 scores from TMEM, reduces their max and min, forms
-//              the E4M3 codes of P~ * 448 32 keys at a time (scores re-read from
-//              TMEM, so only 32 are live next to the exp2 state), writes them
+//              the E4M3 codes of P~ * 448 16 keys at a time (scores re-read from
+//              TMEM, the next 16 loaded while the current 16 are processed, so
+//              only 32 are live next to the exp2 state), writes them
 //              into a 128B-swizzled shared P tile, rescales its row of the O
 //              accumulator in TMEM when its row max moves, and runs the
 //              epilogue.  Two CTAs share an SM.
@@ -100,63 +101,6 @@ __device__ __forceinline__ float int_to_float(uint32_t s) {
   return __int2float_rn(static_cast<int>(s));
 }
 
-// The contract's exponentials for 32 of this thread's keys (biased scores
-// Sb = S + 1.5 * 2^23 as loaded from TMEM; valid counts from the first of
-// them): u = RN(Sb * c + e') with e' = RN(e - 1.5 * 2^23 * c) and
-// e = RN(log2 448 - m_new) (one fused multiply-add per key), y = exp2_fixed_x2(u)
-// -> E4M3 code; the row sum accumulates y.  Every step is a binary32 operation
-// with fixed rounding, so y and its code equal the oracle's bit for bit.
-// kClamp: some u of this warp's tile may be below -126.  pk[w] holds the codes
-// of keys 4w .. 4w+3.  cmul(p) gives the multipliers c and offsets e' of the
-// quarter's keys 2p and 2p+1.
-template <bool kMasked, bool kClamp, class CMul>
-__device__ __forceinline__ void softmax_quarter(const uint32_t (&s)[32], const CMul& cmul, int valid,
-                                                const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t* pk) {
-  // Stage-major over 8 pairs at a time: every step is issued for 8 independent
-  // pairs before the next step, so consecutive instructions do not depend on
-  // each other.
-#pragma unroll
-  for (int h8 = 0; h8 < 2; ++h8) {
-    f32x2_t u[8], xr[8], f[8], p[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int j = 8 * h8 + i;
-      const auto mo = cmul(j);
-      u[i] = x2_fma(x2_pack(s[2 * j], s[2 * j + 1]), mo.c, mo.off);
-    }
-    if (kClamp) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        u[i] = x2_pack(__float_as_uint(fmaxf(x2_lo(u[i]), kExp2Min)), __float_as_uint(fmaxf(x2_hi(u[i]), kExp2Min)));
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) xr[i] = x2_add(u[i], k.round);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = x2_sub(xr[i], k.round);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) f[i] = x2_sub(u[i], f[i]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) p[i] = x2_fma(k.c2, f[i], k.c1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      f32x2_t y = x2_add_exponent(p[i], xr[i]);
-      if (kMasked) {
-        const int j = 8 * h8 + i;
-        const uint32_t lo = 2 * j < valid ? static_cast<uint32_t>(y) : 0u;
-        const uint32_t hi = 2 * j + 1 < valid ? static_cast<uint32_t>(y >> 32) : 0u;
-        y = (static_cast<f32x2_t>(hi) << 32) | lo;
-      }
-      p[i] = y;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) lsum[i & 3] = x2_add(lsum[i & 3], p[i]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) pk[4 * h8 + i] = x2_e4m3x4(p[2 * i], p[2 * i + 1]);
-  }
-}
-
 // Max over the valid keys and min over all keys of 32 biased scores.
 template <bool kMasked>
 __device__ __forceinline__ void chunk_minmax(const uint32_t (&a)[32], int valid, float& mx, float& mn) {
@@ -221,23 +165,84 @@ struct KeyMuls {       // per-key scales of the tile's four 32-key quarters
   }
 };
 
-// The exponential pass over a row's 128 scores in TMEM (taddr), 32 at a time;
-// each chunk's 32 codes go straight to
-// the row's 128B-swizzled P line (16-byte chunk q of row r lives at q ^ (r & 7)).
+// The contract's exponentials for 16 of this thread's keys, pairs 8 h8 .. 8 h8 + 7
+// of a 32-key quarter (biased scores Sb = S + 1.5 * 2^23 as loaded from TMEM;
+// `valid` counts from the quarter's first key): u = RN(Sb * c + e') with
+// e' = RN(e - 1.5 * 2^23 * c) and e = RN(log2 448 - m_new) (one fused
+// multiply-add per key), y = exp2_fixed_x2(u) -> E4M3 code; the row sum
+// accumulates y.  Every step is a binary32 operation with fixed rounding, so y
+// and its code equal the oracle's bit for bit.  kClamp: some u of this warp's
+// tile may be below -126.  pk[w] holds the codes of the chunk's keys 4w .. 4w+3.
+// cmul(p) gives the multipliers c and offsets e' of the quarter's keys 2p and
+// 2p+1.  Stage-major over the 8 pairs: every step is issued for all 8 before
+// the next, so consecutive instructions do not depend on each other.
+template <bool kMasked, bool kClamp, class CMul>
+__device__ __forceinline__ void softmax_eighth(const uint32_t (&s)[16], const CMul& cmul, int h8, int valid,
+                                               const Exp2Consts& k, f32x2_t (&lsum)[4], uint32_t (&pk)[4]) {
+  f32x2_t u[8], xr[8], f[8], p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const auto mo = cmul(8 * h8 + i);
+    u[i] = x2_fma(x2_pack(s[2 * i], s[2 * i + 1]), mo.c, mo.off);
+  }
+  if (kClamp) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      u[i] = x2_pack(__float_as_uint(fmaxf(x2_lo(u[i]), kExp2Min)), __float_as_uint(fmaxf(x2_hi(u[i]), kExp2Min)));
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xr[i] = x2_add(u[i], k.round);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = x2_sub(xr[i], k.round);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = x2_sub(u[i], f[i]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = x2_fma(k.c2, f[i], k.c1);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = x2_fma(p[i], f[i], k.c0);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f32x2_t y = x2_add_exponent(p[i], xr[i]);
+    if (kMasked) {
+      const int j = 8 * h8 + i;
+      const uint32_t lo = 2 * j < valid ? static_cast<uint32_t>(y) : 0u;
+      const uint32_t hi = 2 * j + 1 < valid ? static_cast<uint32_t>(y >> 32) : 0u;
+      y = (static_cast<f32x2_t>(hi) << 32) | lo;
+    }
+    p[i] = y;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) lsum[i & 3] = x2_add(lsum[i & 3], p[i]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) pk[i] = x2_e4m3x4(p[2 * i], p[2 * i + 1]);
+}
+
+// The exponential pass over a row's 128 scores in TMEM (taddr), 16 at a time,
+// the next 16 columns loaded while the current 16 are processed (two 16-word
+// buffers: the same registers as one 32-word chunk); each chunk's 16 codes go
+// straight to the row's 128B-swizzled P line (16-byte chunk q of row r lives at
+// q ^ (r & 7)).
 // kSlow: masked keys or clamped exponents.  muls(qq) gives quarter qq's multipliers.
 template <bool kSlow, class Muls>
 __device__ __forceinline__ void exp_pass(uint32_t taddr, const Muls& muls, int valid,
                                          const Exp2Consts& ek, f32x2_t (&lsum)[4], uint8_t* prow, int row) {
+  uint32_t ra[16], rb[16];
+  tmem_ld16(taddr, ra);
+  tmem_wait_ld();
+  reg_fence16(ra);
 #pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    uint32_t cur[32];
-    tmem_ld32(taddr + 32 * qq, cur);
-    tmem_wait_ld();
-    reg_fence(cur);
-    uint32_t pk[8];
-    softmax_quarter<kSlow, kSlow>(cur, muls(qq), valid - 32 * qq, ek, lsum, pk);
-    *reinterpret_cast<uint4*>(prow + ((2 * qq) ^ (row & 7)) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<uint4*>(prow + ((2 * qq + 1) ^ (row & 7)) * 16) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  for (int c = 0; c < 8; ++c) {
+    uint32_t (&cur)[16] = (c & 1) ? rb : ra;
+    uint32_t (&nxt)[16] = (c & 1) ? ra : rb;
+    if (c < 7) tmem_ld16(taddr + 16 * (c + 1), nxt);
+    const int qq = c >> 1;
+    uint32_t pk[4];
+    softmax_eighth<kSlow, kSlow>(cur, muls(qq), c & 1, valid - 32 * qq, ek, lsum, pk);
+    *reinterpret_cast<uint4*>(prow + (c ^ (row & 7)) * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    if (c < 7) {
+      tmem_wait_ld();
+      reg_fence16(nxt);
+    }
   }
 }
 
