@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
 EXPORTED = ("sage_npad", "sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_fwd",
             "sage_check", "sage_set_wait_timeout_ns", "sage_selftest_wait_timeout", "sage_last_error",
             "sage_quant_qk_static", "sage_quant_qk_normrope", "sage_fp8_quant_rows", "sage_fp8_linear",
-            "sage_quant_qkv")
+            "sage_quant_qkv", "sage_attn_fwd_p_codes")
 QK_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -76,6 +76,9 @@ _lib.sage_quant_v.restype = ctypes.c_int
 _lib.sage_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, SageShape, ctypes.c_float, _vp, ctypes.c_int,
                                _vp, _vp]
 _lib.sage_attn_fwd.restype = ctypes.c_int
+_lib.sage_attn_fwd_p_codes.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, SageShape, ctypes.c_float, _vp,
+                                       ctypes.c_int, _vp, _vp, _vp]
+_lib.sage_attn_fwd_p_codes.restype = ctypes.c_int
 _lib.sage_check.argtypes = [_vp]
 _lib.sage_check.restype = ctypes.c_int
 _lib.sage_set_wait_timeout_ns.argtypes = [ctypes.c_int64]
@@ -204,6 +207,15 @@ def sage_attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean
     _ok(_lib.sage_attn_fwd(_ptr(q_codes), _ptr(q_scale), _ptr(k_codes), _ptr(k_scale), _ptr(v_codes_t),
                            _ptr(v_scale), _ptr(v_mean), shape, float(sm_scale), _ptr(out), int(bool(out_fp32)),
                            _ptr(lse), _stream(stream)), "sage_attn_fwd")
+
+
+def sage_attn_fwd_p_codes(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, shape, sm_scale, out,
+                          out_fp32, p_codes, lse=None, stream=None):
+    """sage_attn_fwd plus the E4M3 codes of P in p_codes (uint8 [B*H, N, npad(N)]); a diagnostic."""
+    _ok(_lib.sage_attn_fwd_p_codes(_ptr(q_codes), _ptr(q_scale), _ptr(k_codes), _ptr(k_scale), _ptr(v_codes_t),
+                                   _ptr(v_scale), _ptr(v_mean), shape, float(sm_scale), _ptr(out),
+                                   int(bool(out_fp32)), _ptr(lse), _ptr(p_codes), _stream(stream)),
+        "sage_attn_fwd_p_codes")
 
 
 def sage_check(stream=None) -> None:

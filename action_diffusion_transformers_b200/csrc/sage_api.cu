@@ -99,6 +99,18 @@ sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullpt
         e = cudaFuncSetAttribute(sage::sage_attn_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::AttnSmem<64>::kAlloc);
       if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_p_codes_kernel<128, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, sage::AttnSmem<128>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_p_codes_kernel<64, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, sage::AttnSmem<64>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_p_codes_kernel<128, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, sage::AttnSmem<128>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::sage_attn_p_codes_kernel<64, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, sage::AttnSmem<64>::kAlloc);
+      if (e == cudaSuccess)
         e = cudaFuncSetAttribute(sage::v_codes_tma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::VbSmem<128>::kAlloc);
       if (e == cudaSuccess)
@@ -583,10 +595,11 @@ sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t, float*
   return launch_check("sage_quant_v launch");
 }
 
-sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
-                          const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
-                          const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32, float* lse,
-                          sage_stream_t stream) {
+// sage_attn_fwd, and with p_codes set its diagnostic form sage_attn_fwd_p_codes.
+static sage_status attn_launch(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
+                               const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
+                               const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32,
+                               float* lse, uint8_t* p_codes, sage_stream_t stream) {
   int64_t ts;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
@@ -634,10 +647,26 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   prm.out_fp32 = out_fp32 ? 1 : 0;
   prm.q_tok = s.q_gran != SAGE_GRAN_BLOCK64;
   prm.timeout_ns = g_timeout_ns.load();
+  prm.p_codes = p_codes;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(static_cast<unsigned>(Npad / sage::kBM), s.H, s.B);
   (void)sm_count;
   const bool k_tok = s.k_gran != SAGE_GRAN_BLOCK64;
+  if (p_codes) {
+    if (s.D == 128 && !k_tok)
+      sage::sage_attn_p_codes_kernel<128, false>
+          <<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+    else if (s.D == 128)
+      sage::sage_attn_p_codes_kernel<128, true>
+          <<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+    else if (!k_tok)
+      sage::sage_attn_p_codes_kernel<64, false>
+          <<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+    else
+      sage::sage_attn_p_codes_kernel<64, true>
+          <<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+    return launch_check("sage_attn_fwd_p_codes launch");
+  }
   if (s.D == 128 && !k_tok)
     sage::sage_attn_kernel<128, false><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
   else if (s.D == 128)
@@ -647,6 +676,23 @@ sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int
   else
     sage::sage_attn_kernel<64, true><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
   return launch_check("sage_attn_fwd launch");
+}
+
+sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
+                          const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
+                          const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32, float* lse,
+                          sage_stream_t stream) {
+  return attn_launch(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, s, sm_scale, out, out_fp32,
+                     lse, nullptr, stream);
+}
+
+sage_status sage_attn_fwd_p_codes(const int8_t* q_codes, const float* q_scale, const int8_t* k_codes,
+                                  const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
+                                  const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32,
+                                  float* lse, uint8_t* p_codes, sage_stream_t stream) {
+  SAGE_NEED(p_codes, "p_codes");
+  return attn_launch(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, s, sm_scale, out, out_fp32,
+                     lse, p_codes, stream);
 }
 
 sage_status sage_fp8_quant_rows(const void* x, int R, int K, int64_t ld, uint8_t* codes, float* scale,

@@ -84,6 +84,7 @@ struct AttnParams {
   int out_fp32;
   int q_tok;              // q_scale holds one scale per token
   int64_t timeout_ns;
+  uint8_t* p_codes;       // [B*H, N, Npad] E4M3 codes of P (sage_attn_p_codes_kernel only)
 };
 
 enum : int { kBarQ = 0, kBarKFull = 1, kBarKEmpty = 3, kBarVFull = 5, kBarVEmpty = 7, kBarSFull = 9,
@@ -290,8 +291,9 @@ __device__ __forceinline__ f32x2_t keywise_exp_pass(uint32_t taddr, float qs, fl
 // tile's K scales differ inside a 64-key half, so every key gets its own
 // multiplier (and the exponent is always clamped); the two instantiations are
 // separate code paths, so the rare per-key tiles leave the register allocation
-// of the common tiles alone.
-template <int D>
+// of the common tiles alone.  kDumpP: also copy the row's finished P line to
+// pdump (the diagnostic kernel).
+template <int D, bool kDumpP>
 struct SoftmaxTile {
   uint64_t* bars;
   volatile int* abort_flag;
@@ -300,6 +302,7 @@ struct SoftmaxTile {
   float qs, sl2e;
   const float* ks;       // per-key K scales of the head (per-key tiles only)
   uint8_t* prow;         // this row of the shared P tile
+  uint8_t* pdump;        // kDumpP: this row's line of the P-code output (null past N)
   int row;
   float& m;              // running row max of t
   float& l;              // running row sum of P~ * 448
@@ -361,6 +364,14 @@ struct SoftmaxTile {
       exp_pass<false>(ts, HalfMuls{c0, c1, off0, off1}, kBN, ek, lsum, prow, row);
     else
       exp_pass<true>(ts, HalfMuls{c0, c1, off0, off1}, valid, ek, lsum, prow, row);
+    if constexpr (kDumpP) {
+      // The thread's own P line, unswizzled: keys j * 128 + 16 c .. + 15 in chunk c.
+      if (pdump != nullptr) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          reinterpret_cast<uint4*>(pdump + j * kBN)[c] = *reinterpret_cast<const uint4*>(prow + (c ^ (row & 7)) * 16);
+      }
+    }
     // Re-seed S with the bias for the next tile's MMA, then release the buffer.
     tmem_fill64(ts, kSBiasBits);
     tmem_fill64(ts + 64, kSBiasBits);
@@ -395,10 +406,11 @@ struct SoftmaxTile {
 // scales).  A tile whose K scales are equal within each 64-key half (the usual
 // case) runs exactly as with 64-token blocks; any other tile takes per-key
 // multipliers and always clamps.
-template <int D, bool kKTok>
-__global__ void __launch_bounds__(kAttnThreads, 2)
-    sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+// kDumpP: the diagnostic form, which also writes every E4M3 code of P to
+// prm.p_codes; the product kernel is the kDumpP = false instantiation.
+template <int D, bool kKTok, bool kDumpP>
+__device__ __forceinline__ void attn_cta(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                         const AttnParams& prm) {
   using L = AttnSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -557,7 +569,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&bars[kBarSEmpty]);
-    SoftmaxTile<D> tile{bars, abort_flag, tmo, ts, to, qs, sl2e, ks, sP + row * 128, row, m, l};
+    uint8_t* pdump = nullptr;
+    if constexpr (kDumpP) {
+      if (qt * kBM + row < prm.N) pdump = prm.p_codes + (static_cast<int64_t>(bh) * prm.N + qt * kBM + row) * prm.Npad;
+    }
+    SoftmaxTile<D, kDumpP> tile{bars, abort_flag, tmo, ts, to, qs, sl2e, ks, sP + row * 128, pdump, row, m, l};
     for (int j = 0; j < nkv; ++j) {
       const int valid = min(kBN, prm.N - j * kBN);   // valid keys in this tile
       float c0, c1;
@@ -642,6 +658,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+template <int D, bool kKTok>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+  attn_cta<D, kKTok, false>(tm_q, tm_k, tm_v, prm);
+}
+
+// The same attention, plus the E4M3 code of every P~ * 448 at
+// prm.p_codes[(bh * N + row) * Npad + key] (keys past N: 0).  For tests.
+template <int D, bool kKTok>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    sage_attn_p_codes_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+  attn_cta<D, kKTok, true>(tm_q, tm_k, tm_v, prm);
 }
 
 }  // namespace sage

@@ -242,6 +242,26 @@ SAGE_API sage_status sage_attn_fwd(const int8_t* q_codes, const float* q_scale,
                           sage_stream_t stream);
 
 /*
+ * sage_attn_fwd_p_codes - sage_attn_fwd that also writes out the E4M3 codes of
+ * P, so that a test can compare them with a reference one by one.  A
+ * diagnostic: the same attention (out and lse as sage_attn_fwd's, bit for
+ * bit), slower by the extra stores.
+ *
+ * out: p_codes  uint8 [B*H, N, sage_npad(N)], caller-owned, 16-byte aligned:
+ *      the code of y = P~ * 448 for key j of query row i of head b*H + h is at
+ *      ((b*H + h) * N + i) * sage_npad(N) + j, formed in key j's 128-key tile
+ *      against that tile's running max; keys j >= N hold 0.
+ * Errors: those of sage_attn_fwd; SAGE_ERR_INVALID_ARG for a NULL p_codes,
+ * SAGE_ERR_ALIGNMENT when it is not 16-byte aligned.
+ */
+SAGE_API sage_status sage_attn_fwd_p_codes(const int8_t* q_codes, const float* q_scale,
+                          const int8_t* k_codes, const float* k_scale,
+                          const uint8_t* v_codes_t, const float* v_scale,
+                          const float* v_mean, sage_shape s, float sm_scale,
+                          void* out, int out_fp32, float* lse, uint8_t* p_codes,
+                          sage_stream_t stream);
+
+/*
  * sage_fp8_quant_rows - per-row E4M3 quantization of a BF16 matrix, for the
  * activations (one scale per token) and, offline, the weights (one scale per
  * output row) of sage_fp8_linear.  ("FLUX.3 Action RTX 5090 report", 02

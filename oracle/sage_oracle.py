@@ -337,7 +337,7 @@ def _identity(x):
 
 
 def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2_alpha, quant_p,
-                 log2_p_unit, two_pass=False, s_bias=0.0):
+                 log2_p_unit, two_pass=False, s_bias=0.0, p_codes=None):
     """Online-softmax attention over 128-key tiles for one (b, h).
 
     S         [R, >= n_keys] float64: exact score numerators (INT32 dot
@@ -377,6 +377,9 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
     amount, at most half an ulp of B * c (below 1.5 c, under two units of the
     integer score).
     two_pass: m is the final row max from the start (alpha = 1 throughout).
+    p_codes: optional uint8 array [R, >= n_keys] that receives the E4M3 code
+    of every y (the code P8 stands for), key by key; the arithmetic is the same
+    with or without it.
     Returns (o [R, D], m [R], l [R]).
     """
     R = S.shape[0]
@@ -406,6 +409,8 @@ def _attend_rows(S, col_mult, Vt, out_mult, out_add, n_keys, rn, fma, exp2, exp2
         y = np.asarray(exp2(fma(S[:, j0:j1] + np.float64(s_bias), c_full, e_off)), dtype=np.float64)
         l = rn(rn(l * alpha) + rn(y.sum(axis=1)))
         p8 = quant_p(y)
+        if p_codes is not None:
+            p_codes[:, j0:j1] = e4m3_encode(y.astype(np.float32))
         acc = rn(rn(acc * alpha[:, None]) + rn(p8 @ Vt[:, j0:j1].T))
         m = m_new
     o = np.asarray(fma(rn(acc * out_mult[None, :]), rn(1.0 / l)[:, None], out_add[None, :]),
@@ -431,7 +436,8 @@ def exp2_scale(sm_scale) -> np.float32:
 
 
 def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
-             sm_scale=None, rows=None, heads=None, two_pass=False, want_lse=False):
+             sm_scale=None, rows=None, heads=None, two_pass=False, want_lse=False,
+             want_p_codes=False):
     """A6-A10 on quantized operands; the output is the FP32 attention output.
 
     q_codes, k_codes int8 [B, H, Npad, D]; q_scale, k_scale f32 [B, H, Npad/64]
@@ -447,7 +453,9 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     sm_scale None or <= 0 means 1/sqrt(D).
     rows: optional query-row indices (< N) to evaluate; heads: optional list of
     (b, h) pairs.  Returns float32 [B, R, H, D] (unevaluated heads stay 0),
-    plus lse [B, H, R] (natural log of the softmax denominator) if asked.
+    plus lse [B, H, R] (natural log of the softmax denominator) if asked, plus
+    the E4M3 codes of P, uint8 [B, H, R, N] (key j of row i holds the code of
+    y = P~ * 448 formed in key j's tile), if want_p_codes.
     """
     B, H, Np, D = q_codes.shape
     if sm_scale is None or sm_scale <= 0:
@@ -457,6 +465,7 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
     R = rows.shape[0]
     out = np.zeros((B, R, H, D), dtype=np.float32)
     lse = np.zeros((B, H, R), dtype=np.float32)
+    pc = np.zeros((B, H, R, N), dtype=np.uint8) if want_p_codes else None
     heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     for b, h in heads:
         Qf = q_codes[b, h, rows].astype(np.float64)
@@ -474,10 +483,11 @@ def attn_fwd(q_codes, q_scale, k_codes, k_scale, v_codes_t, v_scale, v_mean, N,
         o, m, l = _attend_rows(S, col_mult, Vt, v_scale[b, h].astype(np.float64),
                                v_mean[b, h].astype(np.float64), N, rn32, fma32, exp2_contract,
                                _exp2_alpha, _e4m3_round_trip, LOG2_P_UNIT, two_pass=two_pass,
-                               s_bias=S_BIAS)
+                               s_bias=S_BIAS, p_codes=None if pc is None else pc[b, h])
         out[b, :, h, :] = o
         lse[b, h] = rn32((m + np.log2(l) - math.log2(E4M3_MAX)) * math.log(2.0))
-    return (out, lse) if want_lse else out
+    res = (out,) + ((lse,) if want_lse else ()) + ((pc,) if want_p_codes else ())
+    return res if len(res) > 1 else out
 
 
 # ----------------------------------------------------------------------------

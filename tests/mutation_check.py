@@ -41,9 +41,11 @@ M = [
  ("sage_oracle.py", "starts.extend(range(a, e, QK_BLOCK))", "starts.extend(range(a, e, 32))"),
  ("sage_oracle.py", "return f64_to_bf16_bits(s / np.float64(N)).reshape(B, H, D)", "return f64_to_bf16_bits(s / np.float64(N - 1)).reshape(B, H, D)"),
  ("sage_oracle.py", "return np.repeat(scale, QK_BLOCK, axis=-1)", "return np.repeat(scale, 128, axis=-1)[..., :Np]"),
+ ("sage_oracle.py", "p_codes[:, j0:j1] = e4m3_encode(y.astype(np.float32))", "p_codes[:, j0:j1] = e4m3_encode((y * 0.5).astype(np.float32))"),
  ("sage_oracle.py", "sl2e = exp2_scale(sm_scale)\n    rows = np.arange(N) if rows is None else np.asarray(rows)\n    out = np.zeros((B, rows.shape[0], H, D), dtype=np.float32)\n    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads\n    for b, h in heads:\n        S = q_codes", "sl2e = np.float32(sm_scale)\n    rows = np.arange(N) if rows is None else np.asarray(rows)\n    out = np.zeros((B, rows.shape[0], H, D), dtype=np.float32)\n    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads\n    for b, h in heads:\n        S = q_codes"),
 ]
-tests = "tests/test_oracle_sage.py tests/test_oracle_numerics.py tests/test_oracle_plain.py tests/test_oracle_granularity.py"
+tests = ("tests/test_oracle_sage.py tests/test_oracle_numerics.py tests/test_oracle_plain.py "
+         "tests/test_oracle_granularity.py tests/test_oracle_p_codes.py")
 caught = 0
 work = tempfile.mkdtemp(prefix='oracle_mutants_')
 for i, (f, a, b) in enumerate(M):

@@ -108,6 +108,11 @@ def test_attn_and_v_validation(adt):
     assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, None, 0, None, None) == 1
     assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, float("nan"), FAKE, 0, None, None) == 1
     assert L.sage_attn_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, FAKE, 0, FAKE + 2, None) == 3
+    # the diagnostic form: its P-code output is required and 16-byte aligned
+    assert L.sage_attn_fwd_p_codes(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, FAKE, 0, None, None,
+                                   None) == 1
+    assert L.sage_attn_fwd_p_codes(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s, 0.0, FAKE, 0, None, FAKE + 8,
+                                   None) == 3
     assert L.sage_quant_v(FAKE, s, None, FAKE, FAKE, 0x100000, 1 << 40, None) == 1
     assert L.sage_quant_v(FAKE, adt.make_shape(1, 256, 2, 128, 200), FAKE, FAKE, FAKE, 0x100000, 1 << 40,
                           None) == 1
