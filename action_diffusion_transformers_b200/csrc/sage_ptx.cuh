@@ -389,12 +389,16 @@ __device__ __forceinline__ f32x2_t x2_pack(uint32_t lo, uint32_t hi) {
 __device__ __forceinline__ float x2_lo(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
 __device__ __forceinline__ float x2_hi(f32x2_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 // Per 32-bit word: bits(p) + (bits(xr) << 23), i.e. the integer in the low bits
-// of xr added to the exponent field of p.
+// of xr added to the exponent field of p.  The shift is written as a funnel
+// shift of (xr : 0): a plain shl followed by the add is fused by the compiler
+// into an integer multiply-add, which issues on the FMA pipe that the
+// exponential pass saturates; in this form the shift and add stay on the
+// integer ALU pipe (one instruction per word, measured).
 __device__ __forceinline__ f32x2_t x2_add_exponent(f32x2_t p, f32x2_t xr) {
   f32x2_t d;
-  asm("{.reg .b32 pl, ph, xl, xh;\n\t"
-      "mov.b64 {pl, ph}, %1;\n\tmov.b64 {xl, xh}, %2;\n\t"
-      "shl.b32 xl, xl, 23;\n\tshl.b32 xh, xh, 23;\n\t"
+  asm("{.reg .b32 pl, ph, xl, xh, z;\n\t"
+      "mov.b64 {pl, ph}, %1;\n\tmov.b64 {xl, xh}, %2;\n\tmov.b32 z, 0;\n\t"
+      "shf.l.clamp.b32 xl, z, xl, 23;\n\tshf.l.clamp.b32 xh, z, xh, 23;\n\t"
       "add.u32 pl, pl, xl;\n\tadd.u32 ph, ph, xh;\n\t"
       "mov.b64 %0, {pl, ph};}"
       : "=l"(d) : "l"(p), "l"(xr));

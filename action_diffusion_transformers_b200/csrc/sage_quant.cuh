@@ -13,6 +13,7 @@
 // a 16-byte vector for the inputs.  Reductions use a fixed order, so repeated
 // calls give identical bytes.
 #pragma once
+#include <type_traits>
 #include "sage_ptx.cuh"
 
 namespace sage {
@@ -63,12 +64,6 @@ __device__ __forceinline__ f32x2_t x2_of(float lo, float hi) {
   return x2_pack(__float_as_uint(lo), __float_as_uint(hi));
 }
 
-// RN_bf16 of both halves (one packed conversion), returned as binary32.
-__device__ __forceinline__ f32x2_t x2_bf16_round(f32x2_t v) {
-  const __nv_bfloat162 b = __floats2bfloat162_rn(x2_lo(v), x2_hi(v));
-  return x2_of(__low2float(b), __high2float(b));
-}
-
 // Both halves RN_bf16, packed (low half = lo).
 __device__ __forceinline__ uint32_t bf16x2_round(f32x2_t v) {
   uint32_t d;
@@ -89,9 +84,12 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
 // the warp executes this call.  Rows past the data hold zeros and stay zero.
 // The root and reciprocal of row t are formed once, by lane t of the row's
 // lanes, and shuffled out.  cs[t], sn[t]: cos / sin of row t's pairs
-// d0/2 .. d0/2+3.  Products run in f32x2 pairs: the rotation of pair (a, b)
-// is (c*a, s*a) + (-s*b, c*b), each product rounded, then one rounded add per
-// half (RN(-(s*b)) = -RN(s*b), so the first half is RN(RN(c*a) - RN(s*b))).
+// d0/2 .. d0/2+3.  The rotation takes two neighbouring pairs p, p+1 at a time,
+// so that each f32x2 product has as halves the same step of the two pairs:
+// with a = (a_p, a_p+1), b = (b_p, b_p+1), c = (c_p, c_p+1), s = (s_p, s_p+1)
+// (c and s are adjacent words of the tables' float4s) the products are c*a,
+// s*b, s*a and c*b, each rounded, then a' = RN(RN(c*a) - RN(s*b)) and
+// b' = RN(RN(s*a) + RN(c*b)) per pair.
 template <int kRows, int kL>
 __device__ __forceinline__ void norm_rope_rows(float (&x)[kRows][8], const float (&w)[8], float eps,
                                                const float4 (&cs)[kRows], const float4 (&sn)[kRows]) {
@@ -122,20 +120,28 @@ __device__ __forceinline__ void norm_rope_rows(float (&x)[kRows][8], const float
 #pragma unroll
   for (int t = 0; t < kRows; ++t) {
     const f32x2_t r2 = x2_splat(__shfl_sync(0xFFFFFFFFu, rl, base + t));
-    const float c[4] = {cs[t].x, cs[t].y, cs[t].z, cs[t].w};
-    const float s[4] = {sn[t].x, sn[t].y, sn[t].z, sn[t].w};
+    uint32_t zb[4];                       // z of pair p as packed BF16 (low half = even channel)
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const uint32_t y = bf16x2_round(x2_mul(x2_of(x[t][2 * p], x[t][2 * p + 1]), r2));
-      const uint32_t zb = bf16x2_mul(y, w2[p]);
-      const f32x2_t z = x2_of(__uint_as_float(zb << 16), __uint_as_float(zb & 0xFFFF0000u));
-      const f32x2_t t1 = x2_mul(x2_of(c[p], s[p]), x2_splat(x2_lo(z)));
-      const f32x2_t t2 = x2_mul(x2_of(-s[p], c[p]), x2_splat(x2_hi(z)));
+      zb[p] = bf16x2_mul(y, w2[p]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t z0 = zb[2 * h], z1 = zb[2 * h + 1];
+      const f32x2_t a = x2_pack(z0 << 16, z1 << 16);
+      const f32x2_t b = x2_pack(z0 & 0xFFFF0000u, z1 & 0xFFFF0000u);
+      const f32x2_t c = h == 0 ? x2_of(cs[t].x, cs[t].y) : x2_of(cs[t].z, cs[t].w);
+      const f32x2_t s = h == 0 ? x2_of(sn[t].x, sn[t].y) : x2_of(sn[t].z, sn[t].w);
+      const f32x2_t ca = x2_mul(c, a), sb = x2_mul(s, b), sa = x2_mul(s, a), cb = x2_mul(c, b);
       // Scalar adds: the compiler fuses an f32x2 multiply into a following
       // f32x2 add (one rounding fewer), but never a product into __fadd_rn.
-      const f32x2_t o = x2_bf16_round(x2_of(__fadd_rn(x2_lo(t1), x2_lo(t2)), __fadd_rn(x2_hi(t1), x2_hi(t2))));
-      x[t][2 * p] = x2_lo(o);
-      x[t][2 * p + 1] = x2_hi(o);
+      const uint32_t o0 = bf16x2_round(x2_of(__fsub_rn(x2_lo(ca), x2_lo(sb)), __fadd_rn(x2_lo(sa), x2_lo(cb))));
+      const uint32_t o1 = bf16x2_round(x2_of(__fsub_rn(x2_hi(ca), x2_hi(sb)), __fadd_rn(x2_hi(sa), x2_hi(cb))));
+      x[t][4 * h] = __uint_as_float(o0 << 16);
+      x[t][4 * h + 1] = __uint_as_float(o0 & 0xFFFF0000u);
+      x[t][4 * h + 2] = __uint_as_float(o1 << 16);
+      x[t][4 * h + 3] = __uint_as_float(o1 & 0xFFFF0000u);
     }
   }
 }
@@ -240,17 +246,25 @@ __global__ void __launch_bounds__(128) colstats_normrope(const uint16_t* __restr
 #pragma unroll
   for (int i = 0; i < 8; ++i) s[i] = 0.0;
   constexpr int kRows = 4;                 // rows (and their table entries) in flight
+  // A full 64-row block of an active lane loads without guards and zero fills.
+  const bool full = active && n1 - n0 == kSumBlock;
   for (int n = n0; n < n1; n += kRows) {
     uint4 raw[kRows];
     float4 cs[kRows], sn[kRows];
+    auto load_rows = [&](auto guarded) {
 #pragma unroll
-    for (int t = 0; t < kRows; ++t) {
-      const bool ok = active && n + t < n1;
-      const int64_t tab = static_cast<int64_t>(n + t) * (D / 2) + d0 / 2;
-      raw[t] = ok ? ld_nc_16(p + static_cast<int64_t>(n + t - n0) * tok_stride) : make_uint4(0u, 0u, 0u, 0u);
-      cs[t] = ok ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
-      sn[t] = ok ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+      for (int t = 0; t < kRows; ++t) {
+        const bool ok = !decltype(guarded)::value || (active && n + t < n1);
+        const int64_t tab = static_cast<int64_t>(n + t) * (D / 2) + d0 / 2;
+        raw[t] = ok ? ld_nc_16(p + static_cast<int64_t>(n + t - n0) * tok_stride) : make_uint4(0u, 0u, 0u, 0u);
+        cs[t] = ok ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sn[t] = ok ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    };
+    if (full)
+      load_rows(std::false_type{});
+    else
+      load_rows(std::true_type{});
     float f[kRows][8];
 #pragma unroll
     for (int t = 0; t < kRows; ++t) unpack8(raw[t], f[t]);
@@ -410,8 +424,10 @@ __device__ __forceinline__ int rne_small(float y) {
 }
 
 // kNR: Q and K rows first go through QK RMSNorm + RoPE (norm_rope_rows); that
-// variant takes one 64-token block per CTA (4 rows per thread), so that two
-// CTAs fit an SM and one's loads overlap the other's reduction and stores.
+// variant takes one 64-token block per CTA (4 rows per thread), so that
+// several CTAs share an SM and one's loads overlap the others' reductions and
+// stores.  Both variants run three CTAs per SM (80 registers; the kNR one
+// spills a few bytes there and was measured faster than two CTAs at 99).
 template <int D, bool kNR>
 __device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint16_t* __restrict__ q,
                                               const uint16_t* __restrict__ k, int N, int B, int H, int Npad,
@@ -445,17 +461,26 @@ __device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint
   }
   uint4 raw[kTPT];
   float4 cs[kNR ? kTPT : 1], sn[kNR ? kTPT : 1];
+  // Rows past N read as zeros; a CTA whose rows are all below N (every one but
+  // a ragged last tile) loads without the guards and their zero fills.
+  auto load_rows = [&](auto guarded) {
 #pragma unroll
-  for (int t = 0; t < kTPT; ++t) {
-    const int n = tile * kTokens + r0 + t * kRPP;
-    raw[t] = n < N ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
-                   : make_uint4(0u, 0u, 0u, 0u);
-    if constexpr (kNR) {
-      const int64_t tab = static_cast<int64_t>(n) * (D / 2) + d0 / 2;
-      cs[t] = n < N ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
-      sn[t] = n < N ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < kTPT; ++t) {
+      const int n = tile * kTokens + r0 + t * kRPP;
+      const bool ok = !decltype(guarded)::value || n < N;
+      raw[t] = ok ? ld_nc_16(src + (static_cast<int64_t>(b) * N + n) * tok_stride + h * D + d0)
+                  : make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (kNR) {
+        const int64_t tab = static_cast<int64_t>(n) * (D / 2) + d0 / 2;
+        cs[t] = ok ? ld_nc_f4(nr.cos + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+        sn[t] = ok ? ld_nc_f4(nr.sin + tab) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
-  }
+  };
+  if ((tile + 1) * kTokens <= N)
+    load_rows(std::false_type{});
+  else
+    load_rows(std::true_type{});
   float x[kTPT][8];
   float amax[2] = {0.f, 0.f};
 #pragma unroll
@@ -532,7 +557,7 @@ __device__ __forceinline__ void qk_block_body(int bx, int by, int bz, const uint
 }
 
 template <int D, bool kNR = false>
-__global__ void __launch_bounds__(256, kNR ? 2 : 3) qk_block_quant(const uint16_t* __restrict__ q,
+__global__ void __launch_bounds__(256, 3) qk_block_quant(const uint16_t* __restrict__ q,
                                                       const uint16_t* __restrict__ k, int N, int B, int H,
                                                       int Npad, int64_t tok_stride,
                                                       const uint16_t* __restrict__ k_mean,
