@@ -6,7 +6,9 @@
 //  fp8_quant_rows_kernel  one CTA per row: absmax, scale = RN(amax/448),
 //                         inv = RN(448/amax), codes = E4M3(RN(x * inv)).
 //  fp8_gemm_kernel        persistent, one CTA per SM over 128 x 256 output
-//                         (or 128 x 192) tiles.  Warp 0 issues TMA loads of
+//                         (or 128 x 192) tiles; when the last wave would be
+//                         mostly empty, its tiles are split into 2 or 4
+//                         narrower column blocks, so that more SMs share it.  Warp 0 issues TMA loads of
 //                         128 x 128 A and BN x 128 B tiles into a 4- or 5-stage
 //                         ring; warp 1 issues tcgen05.mma kind::f8f6f4 (M 128,
 //                         N BN, K 32) into one of two BN-column TMEM
@@ -112,12 +114,34 @@ struct GemmParams {
   int out_fp32;
   int* err;            // device error word
   int64_t timeout_ns;
+  int tail_start;      // work units below this are whole tiles (unit = tile)
+  int tail_split;      // each tile from tail_start on is this many column blocks (1, 2 or 4)
 };
 
-template <int BN>
+// Work unit -> output block (row tile tm, first column n0, width nw): units
+// below tail_start are whole tiles; unit tail_start + q is column block
+// q % tail_split of tile tail_start + q / tail_split (kTail only).
+template <int BN, bool kTail>
+__device__ __forceinline__ void gemm_unit(const GemmParams& prm, int ntn, int unit, int& tm, int& n0, int& nw) {
+  int tile = unit, sub = 0;
+  nw = BN;
+  if (kTail && unit >= prm.tail_start) {
+    const int q = unit - prm.tail_start;
+    tile = prm.tail_start + q / prm.tail_split;
+    sub = q % prm.tail_split;
+    nw = BN / prm.tail_split;
+  }
+  tm = tile / ntn;
+  n0 = (tile % ntn) * BN + sub * nw;
+}
+
+// tm_b_tail: the W map with a box of BN / tail_split rows (the column blocks).
+// kTail: the last wave is split (prm.tail_split > 1); without it the kernel
+// runs whole tiles only and never reads tm_b_tail.
+template <int BN, bool kTail>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                    const GemmParams prm) {
+                    const __grid_constant__ CUtensorMap tm_b_tail, const GemmParams prm) {
   using L = GemmSmem<BN>;
   constexpr int kGemmBN = BN;
   constexpr int kGemmStages = L::kStages;
@@ -133,6 +157,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int ntm = (prm.M + kGemmBM - 1) / kGemmBM;
   const int ntn = (prm.N + kGemmBN - 1) / kGemmBN;
   const int ntiles = ntm * ntn;
+  const int nunits = kTail ? prm.tail_start + (ntiles - prm.tail_start) * prm.tail_split : ntiles;
   const int nk = (prm.K + kGemmBK - 1) / kGemmBK;
   const int64_t tmo = prm.timeout_ns;
 
@@ -156,17 +181,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
-      uint32_t it = 0;          // stage uses issued, over all tiles
-      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-        const int tm = tile / ntn;
-        const int tn = tile % ntn;
+      if (kTail) tma_prefetch_desc(&tm_b_tail);
+      uint32_t it = 0;          // stage uses issued, over all units
+      for (int unit = blockIdx.x; unit < nunits && !*abort_flag; unit += gridDim.x) {
+        int tm, n0, nw;
+        gemm_unit<kGemmBN, kTail>(prm, ntn, unit, tm, n0, nw);
+        const CUtensorMap* mb = (!kTail || nw == kGemmBN) ? &tm_b : &tm_b_tail;
+        const uint32_t bytes = static_cast<uint32_t>(L::kABytes + nw * kGemmBK);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = static_cast<int>(it % kGemmStages);
           const uint32_t use = it / kGemmStages;
           if (use > 0 && !mbar_wait_bounded(&bars[L::kEmpty + s], (use - 1) & 1, abort_flag, tmo)) break;
-          mbar_arrive_expect_tx(&bars[L::kFull + s], L::kABytes + L::kBBytes);
+          mbar_arrive_expect_tx(&bars[L::kFull + s], bytes);
           tma_load_2d(smem + L::kA + s * L::kABytes, &tm_a, kb * kGemmBK, tm * kGemmBM, &bars[L::kFull + s]);
-          tma_load_2d(smem + L::kB + s * L::kBBytes, &tm_b, kb * kGemmBK, tn * kGemmBN, &bars[L::kFull + s]);
+          tma_load_2d(smem + L::kB + s * L::kBBytes, mb, kb * kGemmBK, n0, &bars[L::kFull + s]);
         }
       }
       if (*abort_flag) {
@@ -185,10 +213,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdesc = make_idesc(1u, 0u, kGemmBM, kGemmBN);   // F32 <- E4M3 x E4M3
+      const uint32_t idesc_tail = kTail ? make_idesc(1u, 0u, kGemmBM, static_cast<uint32_t>(kGemmBN / prm.tail_split))
+                                        : kIdesc;
       uint32_t it = 0;
       uint32_t acc_it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++acc_it) {
+      for (int unit = blockIdx.x; ok && unit < nunits; unit += gridDim.x, ++acc_it) {
+        const uint32_t idesc = (kTail && unit >= prm.tail_start) ? idesc_tail : kIdesc;
         const uint32_t buf = acc_it & 1;
         const uint32_t use = acc_it >> 1;
         if (use > 0 && !mbar_wait_bounded(&bars[L::kAccEmpty + buf], (use - 1) & 1, abort_flag, tmo)) break;
@@ -205,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t bd = make_sdesc(smem_u32(smem + L::kB + s * L::kBBytes), 1024u, 2u);
 #pragma unroll
           for (int kk = 0; kk < kGemmBK / 32; ++kk)
-            mma_f8_ss(d, ad + 2u * kk, bd + 2u * kk, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_f8_ss(d, ad + 2u * kk, bd + 2u * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&bars[L::kEmpty + s]);
         }
         if (ok) tc_commit(&bars[L::kAccFull + buf]);
@@ -220,23 +251,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int quad = warp & 3;                         // TMEM lanes 32*quad .. +31
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t acc_it = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++acc_it) {
+    for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++acc_it) {
       const uint32_t buf = acc_it & 1;
       // the outcome is made the same in every lane before the warp-collective TMEM loads
       const bool ok = mbar_wait_bounded(&bars[L::kAccFull + buf], (acc_it >> 1) & 1, abort_flag, tmo);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
-      const int tm = tile / ntn;
-      const int tn = tile % ntn;
+      int tm, nb, nw;
+      gemm_unit<kGemmBN, kTail>(prm, ntn, unit, tm, nb, nw);
       const int m = tm * kGemmBM + quad * 32 + lane;
       const float sxm = m < prm.M ? prm.sx[m] : 0.f;
 #pragma unroll 1
-      for (int cb = 0; cb < kGemmBN; cb += 32) {
+      for (int cb = 0; cb < (kTail ? nw : kGemmBN); cb += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + buf * kGemmBN + cb + lane_base, r);
         tmem_wait_ld();
         reg_fence(r);
-        const int n0 = tn * kGemmBN + cb;
+        const int n0 = nb + cb;
         if (n0 >= prm.N) continue;                     // the same for the whole warp
         float y[32];
 #pragma unroll

@@ -117,10 +117,13 @@ sage_status device_setup(int* dev_out, int** err_out, int* sm_count_out = nullpt
         e = cudaFuncSetAttribute(sage::v_codes_tma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::VbSmem<64>::kAlloc);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<256, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::GemmSmem<256>::kAlloc);
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<192>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<256, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 sage::GemmSmem<256>::kAlloc);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sage::fp8_gemm_kernel<192, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  sage::GemmSmem<192>::kAlloc);
       if (e == cudaSuccess && !g_encode) {
         void* fn = nullptr;
@@ -749,9 +752,24 @@ sage_status sage_fp8_linear(const uint8_t* xq, const float* sx, const uint8_t* w
     return static_cast<double>(tiles) / static_cast<double>(waves * sms);
   };
   const int BN = (K <= 4096 && fill(192) * 0.95 > fill(256)) ? 192 : 256;
-  CUtensorMap ta, tb;
+  const int64_t tiles = static_cast<int64_t>((M + sage::kGemmBM - 1) / sage::kGemmBM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  // Last wave: when its R tiles would leave most SMs idle, each becomes
+  // `split` column blocks (4 or 2, so that split * R <= the SMs), which the
+  // whole grid shares.  A column block reads the same A tile for a fraction of
+  // the products, so it takes more than 1 / split of a tile's time; the split
+  // is taken only for 256-wide tiles, where the wave is at most half full and
+  // N is a whole number of tiles.
+  const int64_t rem = tiles % grid;
+  int split = 1;
+  if (BN == 256 && tiles > grid && rem > 0 && 2 * rem <= grid && N % BN == 0) split = 4 * rem <= grid ? 4 : 2;
+  CUtensorMap ta, tb, tb_tail;
   if ((st = encode_2d(&ta, xq, K, M, sage::kGemmBK, sage::kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK) return st;
   if ((st = encode_2d(&tb, wq, K, N, sage::kGemmBK, BN, CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK) return st;
+  if (split == 1)
+    tb_tail = tb;   // not read
+  else if ((st = encode_2d(&tb_tail, wq, K, N, sage::kGemmBK, BN / split, CU_TENSOR_MAP_SWIZZLE_128B)) != SAGE_OK)
+    return st;
   sage::GemmParams prm;
   prm.sx = sx;
   prm.sw = sw;
@@ -762,13 +780,16 @@ sage_status sage_fp8_linear(const uint8_t* xq, const float* sx, const uint8_t* w
   prm.out_fp32 = out_fp32 ? 1 : 0;
   prm.err = err;
   prm.timeout_ns = g_timeout_ns.load();
-  const int64_t tiles = static_cast<int64_t>((M + sage::kGemmBM - 1) / sage::kGemmBM) * ((N + BN - 1) / BN);
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  prm.tail_split = split;
+  prm.tail_start = static_cast<int>(split > 1 ? tiles - rem : tiles);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (BN == 256)
-    sage::fp8_gemm_kernel<256><<<grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs>>>(ta, tb, prm);
+  if (BN == 256 && split > 1)
+    sage::fp8_gemm_kernel<256, true><<<grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs>>>(ta, tb, tb_tail, prm);
+  else if (BN == 256)
+    sage::fp8_gemm_kernel<256, false><<<grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs>>>(ta, tb, tb_tail, prm);
   else
-    sage::fp8_gemm_kernel<192><<<grid, sage::kGemmThreads, sage::GemmSmem<192>::kAlloc, cs>>>(ta, tb, prm);
+    sage::fp8_gemm_kernel<192, false><<<grid, sage::kGemmThreads, sage::GemmSmem<192>::kAlloc, cs>>>(ta, tb, tb_tail,
+                                                                                                    prm);
   return launch_check("sage_fp8_linear launch");
 }
 

@@ -840,7 +840,11 @@ __device__ __forceinline__ void v_quant_body(int bx, int by, int bz, const uint1
       unpack8(raw[t], f);
       float y[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fsub_rn(f[i], mean[i]), inv[i]);
+      for (int i = 0; i < 8; i += 2) {     // RN(RN(v - mean) * inv) on pairs
+        const f32x2_t c = x2_mul(x2_sub(x2_of(f[i], f[i + 1]), x2_of(mean[i], mean[i + 1])), x2_of(inv[i], inv[i + 1]));
+        y[i] = x2_lo(c);
+        y[i + 1] = x2_hi(c);
+      }
       w0 = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
       w1 = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
     }
@@ -1008,7 +1012,11 @@ __global__ void __launch_bounds__(kVbThreads, 2)
           unpack8(*reinterpret_cast<const uint4*>(st + nl * L::kRowBytes + 2 * d0), f);
           float y[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fsub_rn(f[i], mean[i]), inv[i]);
+          for (int i = 0; i < 8; i += 2) {   // RN(RN(v - mean) * inv) on pairs
+            const f32x2_t c = x2_mul(x2_sub(x2_of(f[i], f[i + 1]), x2_of(mean[i], mean[i + 1])), x2_of(inv[i], inv[i + 1]));
+            y[i] = x2_lo(c);
+            y[i + 1] = x2_hi(c);
+          }
           w0 = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
           w1 = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
         }

@@ -7,7 +7,9 @@ FP32 summation order meets: |y - y_ref| <= (K * 2^-24 * sum_k |x_k w_k|) * sx
 * sw (the accumulation) + 2 ulp(y) (the two rounded scale products on each
 side).  The BF16 output equals RN_bf16 of the FP32 output bit for bit.
 Shapes cover one tile, ragged M / N / K tails, several waves of the persistent
-grid, and a full-size projection of the action-DiT workload (sampled rows).
+grid, a last wave split into 4 and into 2 column blocks per tile, and full-size
+projections of the action-DiT workload (sampled rows; the MLP down-projection
+splits its last wave).
 """
 import numpy as np
 import pytest
@@ -64,7 +66,10 @@ def test_quant_rows_bit_exact(adt, R, K, ld):
     assert np.array_equal(scale.cpu().numpy().view(np.uint32), rs.view(np.uint32))
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 264, 272), (1000, 1536, 1024), (130, 8, 4096)])
+# (4736, 1280, 4224): 185 tiles of 128 x 256 on 148 SMs, the last 37 as 4 column blocks each;
+# (6656, 1024, 4224): 208 tiles, the last 60 as 2 column blocks each.
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 264, 272), (1000, 1536, 1024), (130, 8, 4096),
+                                   (4736, 1280, 4224), (6656, 1024, 4224)])
 def test_fp8_linear_parity(adt, M, N, K):
     x, w = _inputs(M, N, K, seed=M + N + K)
     xq, sx = _quant(adt, x)
@@ -83,16 +88,19 @@ def test_fp8_linear_parity(adt, M, N, K):
 
 
 @pytest.mark.slow
-def test_fp8_linear_full_size_sampled(adt):
-    """An MLP up-projection of the action-DiT workload: 8192 tokens x 3072 -> 12288."""
-    M, N, K = 8192, 12288, 3072
+@pytest.mark.parametrize("M,N,K", [(8192, 12288, 3072), (8192, 3072, 12288)])
+def test_fp8_linear_full_size_sampled(adt, M, N, K):
+    """The MLP up- and down-projections of the action-DiT workload (8192 tokens,
+    3072 <-> 12288); the down-projection's last wave (tiles of rows 7808 ..
+    8191) runs as column blocks."""
     x, w = _inputs(M, N, K, seed=7)
     xq, sx = _quant(adt, x)
     wq, sw = _quant(adt, w)
     out32 = torch.empty((M, N), dtype=torch.float32, device="cuda")
     adt.sage_fp8_linear(xq, sx, wq, sw, out32)
     adt.sage_check()
-    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], np.random.default_rng(1).choice(M, 60, replace=False)]))
+    rows = np.unique(np.concatenate([[0, 127, 128, 7807, 7808, M - 1], np.random.default_rng(1).choice(M, 60, replace=False),
+                                     np.random.default_rng(2).choice(np.arange(7808, M), 12, replace=False)]))
     xq_h, sx_h, wq_h, sw_h = (t.cpu().numpy() for t in (xq, sx, wq, sw))
     ref = fl.fp8_linear(xq_h[rows], sx_h[rows], wq_h, sw_h)
     y = out32[torch.from_numpy(rows).cuda()].cpu().numpy()

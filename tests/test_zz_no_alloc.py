@@ -7,7 +7,8 @@ library instead of a caller workspace.
 Checked through the C ABI against the existing workspace entry point: two
 calls in a row on different inputs (the second smaller, so scratch left over
 from the first call would show up) must give bit-identical codes, scales and
-K means.  This file is collected last on purpose.
+K means; and directly against the oracle (codes, scales and K means bit for
+bit).  This file is collected last on purpose.
 """
 import ctypes
 
@@ -16,6 +17,7 @@ import pytest
 import torch
 
 import synth
+from oracle import sage_oracle as so
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +59,12 @@ def test_static_scratch_variant_matches_workspace_variant(adt):
         adt.sage_check()
         for key in ref:                           # bit-exact, compared as raw bytes
             assert torch.equal(ref[key].contiguous().view(torch.uint8), got[key].contiguous().view(torch.uint8)), key
+        orc = so.quant_qk(qb, kb)
+        assert np.array_equal(got["q_codes"].cpu().numpy(), orc["q_codes"])
+        assert np.array_equal(got["k_codes"].cpu().numpy(), orc["k_codes"])
+        assert np.array_equal(got["q_scale"].cpu().numpy().view(np.uint32), orc["q_scale"].view(np.uint32))
+        assert np.array_equal(got["k_scale"].cpu().numpy().view(np.uint32), orc["k_scale"].view(np.uint32))
+        assert np.array_equal(got["k_mean"].cpu().view(torch.int16).numpy().view(np.uint16), orc["k_mean"])
 
 
 def test_static_scratch_variant_rejects_oversized_shape(adt):
