@@ -34,6 +34,7 @@ template <int kChunks>
 __global__ void __launch_bounds__(kFqThreads) fp8_quant_rows_kernel(const uint16_t* __restrict__ x, int K,
                                                                     int64_t ld, uint8_t* __restrict__ codes,
                                                                     float* __restrict__ scale) {
+  pdl_enter();
   __shared__ float red[kFqThreads / 32];
   const int r = blockIdx.x;
   const uint16_t* row = x + static_cast<int64_t>(r) * ld;
@@ -142,6 +143,7 @@ template <int BN, bool kTail>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_b_tail, const GemmParams prm) {
+  pdl_enter();
   using L = GemmSmem<BN>;
   constexpr int kGemmBN = BN;
   constexpr int kGemmStages = L::kStages;

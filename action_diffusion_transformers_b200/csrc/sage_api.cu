@@ -216,6 +216,25 @@ sage_status check_ws(const sage_shape& s, const void* ws, size_t ws_bytes, WsLay
   do { if (!(p)) return fail(SAGE_ERR_INVALID_ARG, "%s is NULL", name); \
        if (!aligned16(p)) return fail(SAGE_ERR_ALIGNMENT, "%s is not 16-byte aligned", name); } while (0)
 
+// Launches with programmatic stream serialization allowed: the kernel may be
+// scheduled while the previous kernel in the stream is still running; every
+// kernel of this library begins with pdl_enter(), which waits for that kernel
+// to complete (and its writes to be visible) before anything is read.
+template <typename... KArgs, typename... Args>
+void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 sage_status launch_check(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, what);
@@ -274,11 +293,11 @@ void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const 
     // one 128-token tile per CTA, or one 64-token block with the norm / RoPE
     const dim3 g(Npad / (kNR ? sage::kQKBlock : sage::kTile), s.H, 2 * s.B);
     if (s.D == 128)
-      sage::qk_block_quant<128, kNR><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
-                                                        k_codes, k_scale, nr);
+      pdl_launch(sage::qk_block_quant<128, kNR>, g, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                 q_scale, k_codes, k_scale, nr);
     else
-      sage::qk_block_quant<64, kNR><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
-                                                       k_codes, k_scale, nr);
+      pdl_launch(sage::qk_block_quant<64, kNR>, g, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
+                 q_scale, k_codes, k_scale, nr);
     return;
   }
   sage::SegTable tab;
@@ -295,11 +314,11 @@ void launch_qk_codes(const sage_shape& s, int64_t ts, const uint16_t* qb, const 
     constexpr int GK = decltype(dk)::value;
     if constexpr (GQ != sage::kGranBlock64 || GK != sage::kGranBlock64) {
       if (s.D == 128)
-        sage::qk_group_quant<128, GQ, GK, kNR><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
-                                                                     q_scale, k_codes, k_scale, tab, nr);
+        pdl_launch(sage::qk_group_quant<128, GQ, GK, kNR>, grid, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean,
+                   q_codes, q_scale, k_codes, k_scale, tab, nr);
       else
-        sage::qk_group_quant<64, GQ, GK, kNR><<<grid, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes,
-                                                                    q_scale, k_codes, k_scale, tab, nr);
+        pdl_launch(sage::qk_group_quant<64, GQ, GK, kNR>, grid, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean,
+                   q_codes, q_scale, k_codes, k_scale, tab, nr);
     }
   };
   using G0 = std::integral_constant<int, sage::kGranBlock64>;
@@ -332,8 +351,8 @@ sage_status launch_v_codes(const sage_shape& s, int Npad, int64_t vts, const uin
   if (r != CUDA_SUCCESS) return fail(SAGE_ERR_CUDA, "cuTensorMapEncodeTiled (V rows) failed (%d)", static_cast<int>(r));
   const int total = (Npad / sage::kTile) * s.H * s.B;
   const int grid = std::min(total, 2 * (sm_count > 0 ? sm_count : 148));
-  sage::v_codes_tma<D><<<grid, sage::kVbThreads, sage::VbSmem<D>::kAlloc, cs>>>(
-      tv, vb, s.N, s.H, s.B, Npad, vts, v_mean, vinv, v_codes_t, err, g_timeout_ns.load());
+  pdl_launch(sage::v_codes_tma<D>, grid, sage::kVbThreads, sage::VbSmem<D>::kAlloc, cs, tv, vb, s.N, s.H, s.B, Npad,
+             vts, v_mean, vinv, v_codes_t, err, g_timeout_ns.load());
   return SAGE_OK;
 }
 
@@ -425,10 +444,10 @@ sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_
   const uint16_t* qb = static_cast<const uint16_t*>(q);
   const uint16_t* kb = static_cast<const uint16_t*>(k);
 
-  sage::colstats_partial<false><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum,
-                                                                                    nullptr, nullptr);
-  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
-                                                                static_cast<uint16_t*>(k_mean));
+  pdl_launch(sage::colstats_partial<false>, dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs, kb, s.N, HD, ts, nsb,
+             psum, nullptr, nullptr);
+  pdl_launch(sage::k_mean_finalize, (s.B * HD + 31) / 32, 1024, 0, cs, psum, s.B, s.N, HD, nsb, kmean,
+             static_cast<uint16_t*>(k_mean));
   launch_qk_codes<false>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, sage::NormRopeArgs{}, cs);
   return launch_check("sage_quant_qk launch");
 }
@@ -486,23 +505,23 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   const uint16_t* kb = static_cast<const uint16_t*>(k);
   const uint16_t* vb = static_cast<const uint16_t*>(v);
 
-  sage::colstats_kv<<<dim3(nsb, s.B, 2 * zc), 128, 0, cs>>>(kb, vb, s.N, HD, ts, vts, nsb, zc, psum_k, psum_v, pmin,
-                                                             pmax);
+  pdl_launch(sage::colstats_kv, dim3(nsb, s.B, 2 * zc), 128, 0, cs, kb, vb, s.N, HD, ts, vts, nsb, zc, psum_k, psum_v,
+             pmin, pmax);
   const int nf = (s.B * HD + 31) / 32;
-  sage::finalize_kv<<<2 * nf, 1024, 0, cs>>>(psum_k, psum_v, pmin, pmax, s.B, s.N, HD, nsb, nf, kmean,
-                                              static_cast<uint16_t*>(k_mean), v_mean, v_scale, vinv);
+  pdl_launch(sage::finalize_kv, 2 * nf, 1024, 0, cs, psum_k, psum_v, pmin, pmax, s.B, s.N, HD, nsb, nf, kmean,
+             static_cast<uint16_t*>(k_mean), v_mean, v_scale, vinv);
   // The code passes stay two launches: merged, the V blocks would take the Q/K
   // blocks' register allocation and fit fewer per SM (measured slower).
   const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
   const dim3 gv(Npad / sage::kTile, s.H, s.B);
   if (s.D == 128) {
-    sage::qk_block_quant<128><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
-                                                 k_scale);
+    pdl_launch(sage::qk_block_quant<128>, g, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+               k_codes, k_scale, sage::NormRopeArgs{});
     if ((st = launch_v_codes<128>(s, Npad, vts, vb, v_mean, vinv, v_codes_t, err, sm_count, cs)) != SAGE_OK)
       return st;
   } else {
-    sage::qk_block_quant<64><<<g, 256, 0, cs>>>(qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale, k_codes,
-                                                k_scale);
+    pdl_launch(sage::qk_block_quant<64>, g, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
+               k_codes, k_scale, sage::NormRopeArgs{});
     if ((st = launch_v_codes<64>(s, Npad, vts, vb, v_mean, vinv, v_codes_t, err, sm_count, cs)) != SAGE_OK)
       return st;
   }
@@ -551,11 +570,11 @@ sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s, c
 
   const dim3 sg(nsb, s.B, (HD + 1023) / 1024);
   if (s.D == 128)
-    sage::colstats_normrope<128><<<sg, 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum, a);
+    pdl_launch(sage::colstats_normrope<128>, sg, 128, 0, cs, kb, s.N, HD, ts, nsb, psum, a);
   else
-    sage::colstats_normrope<64><<<sg, 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum, a);
-  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
-                                                                static_cast<uint16_t*>(k_mean));
+    pdl_launch(sage::colstats_normrope<64>, sg, 128, 0, cs, kb, s.N, HD, ts, nsb, psum, a);
+  pdl_launch(sage::k_mean_finalize, (s.B * HD + 31) / 32, 1024, 0, cs, psum, s.B, s.N, HD, nsb, kmean,
+             static_cast<uint16_t*>(k_mean));
   launch_qk_codes<true>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, a, cs);
   return launch_check("sage_quant_qk_normrope launch");
 }
@@ -586,15 +605,15 @@ sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t, float*
   const int Npad = static_cast<int>(npad_of(s.N));
   const uint16_t* vb = static_cast<const uint16_t*>(v);
 
-  sage::colstats_partial<true><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(vb, s.N, HD, ts, nsb, psum,
-                                                                                   pmin, pmax);
-  sage::v_stats_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, pmin, pmax, s.B, s.N, HD, nsb, v_mean,
-                                                                 v_scale, vinv);
+  pdl_launch(sage::colstats_partial<true>, dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs, vb, s.N, HD, ts, nsb, psum,
+             pmin, pmax);
+  pdl_launch(sage::v_stats_finalize, (s.B * HD + 31) / 32, 1024, 0, cs, psum, pmin, pmax, s.B, s.N, HD, nsb, v_mean,
+             v_scale, vinv);
   const dim3 g(Npad / sage::kTile, s.H, s.B);
   if (s.D == 128)
-    sage::v_quant_t<128><<<g, 256, 0, cs>>>(vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
+    pdl_launch(sage::v_quant_t<128>, g, 256, 0, cs, vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
   else
-    sage::v_quant_t<64><<<g, 256, 0, cs>>>(vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
+    pdl_launch(sage::v_quant_t<64>, g, 256, 0, cs, vb, s.N, s.H, Npad, ts, v_mean, vinv, v_codes_t);
   return launch_check("sage_quant_v launch");
 }
 
@@ -657,27 +676,31 @@ static sage_status attn_launch(const int8_t* q_codes, const float* q_scale, cons
   const bool k_tok = s.k_gran != SAGE_GRAN_BLOCK64;
   if (p_codes) {
     if (s.D == 128 && !k_tok)
-      sage::sage_attn_p_codes_kernel<128, false>
-          <<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+      pdl_launch(sage::sage_attn_p_codes_kernel<128, false>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc,
+                 cs, tq, tk, tv, prm);
     else if (s.D == 128)
-      sage::sage_attn_p_codes_kernel<128, true>
-          <<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+      pdl_launch(sage::sage_attn_p_codes_kernel<128, true>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs,
+                 tq, tk, tv, prm);
     else if (!k_tok)
-      sage::sage_attn_p_codes_kernel<64, false>
-          <<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+      pdl_launch(sage::sage_attn_p_codes_kernel<64, false>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs,
+                 tq, tk, tv, prm);
     else
-      sage::sage_attn_p_codes_kernel<64, true>
-          <<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+      pdl_launch(sage::sage_attn_p_codes_kernel<64, true>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs,
+                 tq, tk, tv, prm);
     return launch_check("sage_attn_fwd_p_codes launch");
   }
   if (s.D == 128 && !k_tok)
-    sage::sage_attn_kernel<128, false><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+    pdl_launch(sage::sage_attn_kernel<128, false>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs, tq, tk,
+               tv, prm);
   else if (s.D == 128)
-    sage::sage_attn_kernel<128, true><<<grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs>>>(tq, tk, tv, prm);
+    pdl_launch(sage::sage_attn_kernel<128, true>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs, tq, tk,
+               tv, prm);
   else if (!k_tok)
-    sage::sage_attn_kernel<64, false><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+    pdl_launch(sage::sage_attn_kernel<64, false>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq, tk,
+               tv, prm);
   else
-    sage::sage_attn_kernel<64, true><<<grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs>>>(tq, tk, tv, prm);
+    pdl_launch(sage::sage_attn_kernel<64, true>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq, tk, tv,
+               prm);
   return launch_check("sage_attn_fwd launch");
 }
 
@@ -717,11 +740,11 @@ sage_status sage_fp8_quant_rows(const void* x, int R, int K, int64_t ld, uint8_t
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   const int per = K / 8;
   if (per <= 4 * sage::kFqThreads)
-    sage::fp8_quant_rows_kernel<4><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+    pdl_launch(sage::fp8_quant_rows_kernel<4>, R, sage::kFqThreads, 0, cs, xb, K, lds, codes, scale);
   else if (per <= 8 * sage::kFqThreads)
-    sage::fp8_quant_rows_kernel<8><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+    pdl_launch(sage::fp8_quant_rows_kernel<8>, R, sage::kFqThreads, 0, cs, xb, K, lds, codes, scale);
   else
-    sage::fp8_quant_rows_kernel<16><<<R, sage::kFqThreads, 0, cs>>>(xb, K, lds, codes, scale);
+    pdl_launch(sage::fp8_quant_rows_kernel<16>, R, sage::kFqThreads, 0, cs, xb, K, lds, codes, scale);
   return launch_check("sage_fp8_quant_rows launch");
 }
 
@@ -784,12 +807,14 @@ sage_status sage_fp8_linear(const uint8_t* xq, const float* sx, const uint8_t* w
   prm.tail_start = static_cast<int>(split > 1 ? tiles - rem : tiles);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if (BN == 256 && split > 1)
-    sage::fp8_gemm_kernel<256, true><<<grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs>>>(ta, tb, tb_tail, prm);
+    pdl_launch(sage::fp8_gemm_kernel<256, true>, grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs, ta, tb,
+               tb_tail, prm);
   else if (BN == 256)
-    sage::fp8_gemm_kernel<256, false><<<grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs>>>(ta, tb, tb_tail, prm);
+    pdl_launch(sage::fp8_gemm_kernel<256, false>, grid, sage::kGemmThreads, sage::GemmSmem<256>::kAlloc, cs, ta, tb,
+               tb_tail, prm);
   else
-    sage::fp8_gemm_kernel<192, false><<<grid, sage::kGemmThreads, sage::GemmSmem<192>::kAlloc, cs>>>(ta, tb, tb_tail,
-                                                                                                    prm);
+    pdl_launch(sage::fp8_gemm_kernel<192, false>, grid, sage::kGemmThreads, sage::GemmSmem<192>::kAlloc, cs, ta, tb,
+               tb_tail, prm);
   return launch_check("sage_fp8_linear launch");
 }
 
@@ -820,7 +845,7 @@ sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream)
   int* err;
   sage_status st = device_setup(&dev, &err);
   if (st != SAGE_OK) return st;
-  selftest_wait_kernel<0><<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(timeout_ns, err);
+  pdl_launch(selftest_wait_kernel<0>, 1, 32, 0, reinterpret_cast<cudaStream_t>(stream), timeout_ns, err);
   return launch_check("selftest launch");
 }
 
@@ -860,10 +885,10 @@ sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int
   const uint16_t* qb = static_cast<const uint16_t*>(q);
   const uint16_t* kb = static_cast<const uint16_t*>(k);
   // Every scratch byte read below is written earlier in the same call.
-  sage::colstats_partial<false><<<dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs>>>(kb, s.N, HD, ts, nsb, psum,
-                                                                                    nullptr, nullptr);
-  sage::k_mean_finalize<<<(s.B * HD + 31) / 32, 1024, 0, cs>>>(psum, s.B, s.N, HD, nsb, kmean,
-                                                                static_cast<uint16_t*>(k_mean));
+  pdl_launch(sage::colstats_partial<false>, dim3(nsb, s.B, (HD + 1023) / 1024), 128, 0, cs, kb, s.N, HD, ts, nsb,
+             psum, nullptr, nullptr);
+  pdl_launch(sage::k_mean_finalize, (s.B * HD + 31) / 32, 1024, 0, cs, psum, s.B, s.N, HD, nsb, kmean,
+             static_cast<uint16_t*>(k_mean));
   launch_qk_codes<false>(s, ts, qb, kb, kmean, q_codes, q_scale, k_codes, k_scale, sage::NormRopeArgs{}, cs);
   return launch_check("sage_quant_qk_static launch");
 }

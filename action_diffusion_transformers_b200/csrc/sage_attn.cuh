@@ -664,6 +664,7 @@ template <int D, bool kKTok>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     sage_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+  pdl_enter();
   attn_cta<D, kKTok, false>(tm_q, tm_k, tm_v, prm);
 }
 
@@ -673,6 +674,7 @@ template <int D, bool kKTok>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     sage_attn_p_codes_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+  pdl_enter();
   attn_cta<D, kKTok, true>(tm_q, tm_k, tm_v, prm);
 }
 

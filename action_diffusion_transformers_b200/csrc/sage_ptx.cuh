@@ -7,6 +7,14 @@
 
 namespace sage {
 
+// Programmatic dependent launch: wait until the grids this one depends on have
+// completed and their writes are visible (a no-op when the launch did not allow
+// an early start), then allow the next grid in the stream to be scheduled.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Two binary32 values held in one 64-bit register (first value in the low
 // word), the operand form of the sm_100 add/mul/fma.f32x2 instructions.  The
 // pair never leaves its register between operations, so no moves are needed

@@ -221,6 +221,7 @@ __global__ void __launch_bounds__(128) colstats_partial(const uint16_t* __restri
                                                         int64_t tok_stride, int nsb,
                                                         double* __restrict__ psum,
                                                         float* __restrict__ pmin, float* __restrict__ pmax) {
+  pdl_enter();
   colstats_body<kMinMax>(blockIdx.x, blockIdx.y, blockIdx.z, x, N, HD, tok_stride, nsb, psum, pmin, pmax);
 }
 
@@ -232,6 +233,7 @@ template <int D>
 __global__ void __launch_bounds__(128) colstats_normrope(const uint16_t* __restrict__ x, int N, int HD,
                                                          int64_t tok_stride, int nsb, double* __restrict__ psum,
                                                          const NormRopeArgs nr) {
+  pdl_enter();
   const int c = blockIdx.x;
   const int b = blockIdx.y;
   const int ch0 = (blockIdx.z * blockDim.x + threadIdx.x) * 8;
@@ -365,6 +367,7 @@ __device__ __forceinline__ void k_mean_body(int bx, const double* __restrict__ p
 __global__ void __launch_bounds__(1024) k_mean_finalize(const double* __restrict__ psum, int B, int N, int HD,
                                                         int nsb, uint16_t* __restrict__ mean_ws,
                                                         uint16_t* __restrict__ mean_out) {
+  pdl_enter();
   __shared__ double sh[kSumLanes][33];
   k_mean_body(blockIdx.x, psum, B, N, HD, nsb, mean_ws, mean_out, sh);
 }
@@ -403,6 +406,7 @@ __global__ void __launch_bounds__(1024) v_stats_finalize(const double* __restric
                                                          const float* __restrict__ pmax, int B, int N, int HD,
                                                          int nsb, float* __restrict__ v_mean,
                                                          float* __restrict__ v_scale, float* __restrict__ v_inv) {
+  pdl_enter();
   __shared__ double sh[kSumLanes][33];
   __shared__ float shn[kSumLanes][33];
   __shared__ float shx[kSumLanes][33];
@@ -564,6 +568,7 @@ __global__ void __launch_bounds__(256, 3) qk_block_quant(const uint16_t* __restr
                                                       int8_t* __restrict__ q_codes, float* __restrict__ q_scale,
                                                       int8_t* __restrict__ k_codes,
                                                       float* __restrict__ k_scale, const NormRopeArgs nr = {}) {
+  pdl_enter();
   qk_block_body<D, kNR>(blockIdx.x, blockIdx.y, blockIdx.z, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes,
                         q_scale, k_codes, k_scale, nr);
 }
@@ -785,6 +790,7 @@ __global__ void __launch_bounds__(256, kNR ? 1 : ((kGranQ == kGranSegment64 || k
                    int64_t tok_stride, const uint16_t* __restrict__ k_mean, int8_t* __restrict__ q_codes,
                    float* __restrict__ q_scale, int8_t* __restrict__ k_codes, float* __restrict__ k_scale,
                    const __grid_constant__ SegTable seg, const NormRopeArgs nr = {}) {
+  pdl_enter();
   if (static_cast<int>(blockIdx.z) < B)
     group_quant_cta<D, kGranK, kNR>(true, q, k, N, B, H, Npad, tok_stride, k_mean, q_codes, q_scale, k_codes,
                                     k_scale, seg, nr);
@@ -886,6 +892,7 @@ template <int D>
 __global__ void __launch_bounds__(256) v_quant_t(const uint16_t* __restrict__ v, int N, int H, int Npad,
                                                  int64_t tok_stride, const float* __restrict__ v_mean,
                                                  const float* __restrict__ v_inv, uint8_t* __restrict__ out) {
+  pdl_enter();
   v_quant_body<D>(blockIdx.x, blockIdx.y, blockIdx.z, v, N, H, Npad, tok_stride, v_mean, v_inv, out);
 }
 
@@ -923,6 +930,7 @@ __global__ void __launch_bounds__(kVbThreads, 2)
     v_codes_tma(const __grid_constant__ CUtensorMap tm_v, const uint16_t* __restrict__ v, int N, int H, int B,
                  int Npad, int64_t tok_stride, const float* __restrict__ v_mean, const float* __restrict__ v_inv,
                  uint8_t* __restrict__ out, int* err, int64_t timeout_ns) {
+  pdl_enter();
   using L = VbSmem<D>;
   constexpr int kLPR = D / 8;
   constexpr int kRPP = kVbConsumers / kLPR;
@@ -1071,6 +1079,7 @@ __global__ void __launch_bounds__(128) colstats_kv(const uint16_t* __restrict__ 
                                                    int N, int HD, int64_t k_stride, int64_t v_stride, int nsb,
                                                    int zc, double* __restrict__ psum_k, double* __restrict__ psum_v,
                                                    float* __restrict__ pmin, float* __restrict__ pmax) {
+  pdl_enter();
   const int z = static_cast<int>(blockIdx.z);
   if (z >= zc)
     colstats_body<false>(blockIdx.x, blockIdx.y, z - zc, k, N, HD, k_stride, nsb, psum_k, nullptr, nullptr);
@@ -1087,6 +1096,7 @@ __global__ void __launch_bounds__(1024) finalize_kv(const double* __restrict__ p
                                                     uint16_t* __restrict__ mean_ws, uint16_t* __restrict__ mean_out,
                                                     float* __restrict__ v_mean, float* __restrict__ v_scale,
                                                     float* __restrict__ v_inv) {
+  pdl_enter();
   __shared__ double sh[kSumLanes][33];
   __shared__ float shn[kSumLanes][33];
   __shared__ float shx[kSumLanes][33];
