@@ -220,7 +220,11 @@ sage_status check_ws(const sage_shape& s, const void* ws, size_t ws_bytes, WsLay
 // scheduled while the previous kernel in the stream is still running; every
 // kernel of this library begins with pdl_enter(), which waits for that kernel
 // to complete (and its writes to be visible) before anything is read.
-template <typename... KArgs, typename... Args>
+// kEarly = false: an ordinary launch (after the previous kernel has finished),
+// used for the attention kernel: with its blocks scheduled early beside the
+// last quantization pass it measured 0.35% slower on one B200 and the same on
+// another, for a gain of a few microseconds per step at most.
+template <bool kEarly = true, typename... KArgs, typename... Args>
 void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -231,7 +235,7 @@ void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kEarly ? 1 : 0;
   (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
@@ -676,31 +680,31 @@ static sage_status attn_launch(const int8_t* q_codes, const float* q_scale, cons
   const bool k_tok = s.k_gran != SAGE_GRAN_BLOCK64;
   if (p_codes) {
     if (s.D == 128 && !k_tok)
-      pdl_launch(sage::sage_attn_p_codes_kernel<128, false>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc,
-                 cs, tq, tk, tv, prm);
+      pdl_launch<false>(sage::sage_attn_p_codes_kernel<128, false>, grid, sage::kAttnThreads,
+                        sage::AttnSmem<128>::kAlloc, cs, tq, tk, tv, prm);
     else if (s.D == 128)
-      pdl_launch(sage::sage_attn_p_codes_kernel<128, true>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs,
-                 tq, tk, tv, prm);
+      pdl_launch<false>(sage::sage_attn_p_codes_kernel<128, true>, grid, sage::kAttnThreads,
+                        sage::AttnSmem<128>::kAlloc, cs, tq, tk, tv, prm);
     else if (!k_tok)
-      pdl_launch(sage::sage_attn_p_codes_kernel<64, false>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs,
-                 tq, tk, tv, prm);
+      pdl_launch<false>(sage::sage_attn_p_codes_kernel<64, false>, grid, sage::kAttnThreads,
+                        sage::AttnSmem<64>::kAlloc, cs, tq, tk, tv, prm);
     else
-      pdl_launch(sage::sage_attn_p_codes_kernel<64, true>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs,
-                 tq, tk, tv, prm);
+      pdl_launch<false>(sage::sage_attn_p_codes_kernel<64, true>, grid, sage::kAttnThreads,
+                        sage::AttnSmem<64>::kAlloc, cs, tq, tk, tv, prm);
     return launch_check("sage_attn_fwd_p_codes launch");
   }
   if (s.D == 128 && !k_tok)
-    pdl_launch(sage::sage_attn_kernel<128, false>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs, tq, tk,
-               tv, prm);
+    pdl_launch<false>(sage::sage_attn_kernel<128, false>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs,
+                      tq, tk, tv, prm);
   else if (s.D == 128)
-    pdl_launch(sage::sage_attn_kernel<128, true>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs, tq, tk,
-               tv, prm);
+    pdl_launch<false>(sage::sage_attn_kernel<128, true>, grid, sage::kAttnThreads, sage::AttnSmem<128>::kAlloc, cs,
+                      tq, tk, tv, prm);
   else if (!k_tok)
-    pdl_launch(sage::sage_attn_kernel<64, false>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq, tk,
-               tv, prm);
+    pdl_launch<false>(sage::sage_attn_kernel<64, false>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq,
+                      tk, tv, prm);
   else
-    pdl_launch(sage::sage_attn_kernel<64, true>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq, tk, tv,
-               prm);
+    pdl_launch<false>(sage::sage_attn_kernel<64, true>, grid, sage::kAttnThreads, sage::AttnSmem<64>::kAlloc, cs, tq,
+                      tk, tv, prm);
   return launch_check("sage_attn_fwd launch");
 }
 
