@@ -236,6 +236,8 @@ void pdl_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = kEarly ? 1 : 0;
+  // A failed launch is also recorded as this thread's last CUDA error, which
+  // launch_check() reads after the call's launches.
   (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 

@@ -21,7 +21,12 @@
  *    allocates or frees memory; scratch space is the caller's workspace.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream) and never synchronise.  Device-side wait timeouts are
- *    reported by sage_check().
+ *    reported by sage_check().  The quantization and projection kernels are
+ *    launched with programmatic dependent launch: their blocks may be
+ *    scheduled while the previous kernel on the stream is still running, and
+ *    each waits for that kernel to complete before it reads anything, so
+ *    stream order is kept for every input, including the caller's own
+ *    kernels and copies.
  *  - Arguments are validated on the host before any launch.  On an invalid
  *    argument nothing is launched, the call returns a non-zero sage_status,
  *    and sage_last_error() describes the problem (thread-local string).
