@@ -75,3 +75,37 @@ def test_single_rank_is_identity():
     from action_diffusion_transformers_b200 import sp
     x = torch.randn(1, 8, 2, 4)
     assert sp.seq_to_head(x) is x and sp.head_to_seq(x) is x
+
+
+def _shape_worker(rank: int, world: int, port: int, out_dir: str):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    from action_diffusion_transformers_b200 import sp
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        res = {}
+        # the checks run before any exchange, so every rank refuses alike and no collective is left waiting
+        for name, fn, t in (("heads", sp.seq_to_head, torch.zeros(1, 4, 3, 8, dtype=torch.int16)),
+                            ("tokens", sp.head_to_seq, torch.zeros(1, 5, 2, 8, dtype=torch.int16))):
+            try:
+                fn(t)
+                res[name] = "accepted"
+            except ValueError as e:
+                res[name] = "refused" if f"{world} ranks" in str(e) else "wrong message"
+        with open(os.path.join(out_dir, f"shape{rank}.txt"), "w") as f:
+            f.write(" ".join(f"{k}={v}" for k, v in res.items()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shapes_that_do_not_divide_are_refused(tmp_path):
+    """H (for the gather) and N (for the return) must be multiples of the rank count."""
+    mp.start_processes(_shape_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    for rank in range(2):
+        res = dict(kv.split("=") for kv in open(tmp_path / f"shape{rank}.txt").read().split())
+        assert res == {"heads": "refused", "tokens": "refused"}, (rank, res)
