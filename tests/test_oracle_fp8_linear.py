@@ -5,7 +5,6 @@ the scaled product by power-of-two identities and a closed form."""
 from fractions import Fraction
 
 import numpy as np
-import pytest
 
 import synth
 from oracle import fp8_linear as fl

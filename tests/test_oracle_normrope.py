@@ -6,7 +6,6 @@ rotation, an FP64 restatement within BF16 rounding, and invariances (per-head
 scale, rotation composition) that a wrong axis or a swapped pair would break.
 """
 import numpy as np
-import pytest
 
 import synth
 from oracle import normrope as nr

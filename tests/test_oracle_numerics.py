@@ -9,7 +9,6 @@ import struct
 from fractions import Fraction
 
 import numpy as np
-import pytest
 import torch
 
 from oracle import numerics as nm

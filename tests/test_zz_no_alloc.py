@@ -10,8 +10,6 @@ from the first call would show up) must give bit-identical codes, scales and
 K means; and directly against the oracle (codes, scales and K means bit for
 bit).  This file is collected last on purpose.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
