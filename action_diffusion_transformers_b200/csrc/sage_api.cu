@@ -413,7 +413,7 @@ extern "C" {
 size_t sage_npad(int N) { return N < 1 ? 0 : static_cast<size_t>(npad_of(N)); }
 
 size_t sage_workspace_bytes(sage_shape s) {
-  int64_t ts;
+  int64_t ts = 0;
   if (check_shape(s, &ts) != SAGE_OK) return 0;
   return ws_layout(s).total;
 }
@@ -425,7 +425,7 @@ void sage_set_wait_timeout_ns(int64_t ns) { g_timeout_ns.store(ns > 0 ? ns : 200
 sage_status sage_quant_qk(const void* q, const void* k, sage_shape s, int8_t* q_codes, float* q_scale,
                           int8_t* k_codes, float* k_scale, void* k_mean, void* workspace, size_t ws_bytes,
                           sage_stream_t stream) {
-  int64_t ts;
+  int64_t ts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   SAGE_NEED(q, "q");
@@ -471,7 +471,7 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
     sv.tok_stride = v_tok_stride;
     return sage_quant_v(v, sv, v_codes_t, v_scale, v_mean, workspace, ws_bytes, stream);
   }
-  int64_t ts, vts;
+  int64_t ts = 0, vts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   sage_shape sv = s;
@@ -519,7 +519,6 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
   // The code passes stay two launches: merged, the V blocks would take the Q/K
   // blocks' register allocation and fit fewer per SM (measured slower).
   const dim3 g(Npad / sage::kTile, s.H, 2 * s.B);
-  const dim3 gv(Npad / sage::kTile, s.H, s.B);
   if (s.D == 128) {
     pdl_launch(sage::qk_block_quant<128>, g, 256, 0, cs, qb, kb, s.N, s.B, s.H, Npad, ts, kmean, q_codes, q_scale,
                k_codes, k_scale, sage::NormRopeArgs{});
@@ -537,7 +536,7 @@ sage_status sage_quant_qkv(const void* q, const void* k, const void* v, sage_sha
 sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s, const sage_normrope* nr,
                                    int8_t* q_codes, float* q_scale, int8_t* k_codes, float* k_scale, void* k_mean,
                                    void* workspace, size_t ws_bytes, sage_stream_t stream) {
-  int64_t ts;
+  int64_t ts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   SAGE_NEED(q, "q");
@@ -587,7 +586,7 @@ sage_status sage_quant_qk_normrope(const void* q, const void* k, sage_shape s, c
 
 sage_status sage_quant_v(const void* v, sage_shape s, uint8_t* v_codes_t, float* v_scale, float* v_mean,
                          void* workspace, size_t ws_bytes, sage_stream_t stream) {
-  int64_t ts;
+  int64_t ts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   SAGE_NEED(v, "v");
@@ -628,7 +627,7 @@ static sage_status attn_launch(const int8_t* q_codes, const float* q_scale, cons
                                const float* k_scale, const uint8_t* v_codes_t, const float* v_scale,
                                const float* v_mean, sage_shape s, float sm_scale, void* out, int out_fp32,
                                float* lse, uint8_t* p_codes, sage_stream_t stream) {
-  int64_t ts;
+  int64_t ts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   SAGE_NEED(q_codes, "q_codes");
@@ -858,7 +857,7 @@ sage_status sage_selftest_wait_timeout(int64_t timeout_ns, sage_stream_t stream)
 
 sage_status sage_quant_qk_static(const void* q, const void* k, sage_shape s, int8_t* q_codes, float* q_scale,
                                  int8_t* k_codes, float* k_scale, void* k_mean, sage_stream_t stream) {
-  int64_t ts;
+  int64_t ts = 0;
   sage_status st = check_shape(s, &ts);
   if (st != SAGE_OK) return st;
   SAGE_NEED(q, "q");
